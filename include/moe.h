@@ -1,0 +1,210 @@
+/*
+ * moe.h -- C ABI of the routed mixture-of-experts FFN layer over MXFP4 expert
+ * weights, for NVIDIA B200 (sm_100a).
+ *
+ * What the layer is (the pages describe it; none prints its formulas):
+ *   - DeepSeek-V4-Flash's routed MoE layer: per token only k of E experts run,
+ *     and only the activated experts' weights are read from memory
+ *     (ainews.cool "antirez ds4 DeepSeek Metal inference", section
+ *     技术深度解析: block-sparse matmul over activated experts only).
+ *   - routed experts are stored as MXFP4 ("ds4-ssd" README, "Run SSD Sidecar
+ *     Mode": native package with bit-exact MXFP4 routed experts).  MXFP4 is the
+ *     OCP Microscaling v1.0 format: 32 E2M1 (4-bit) values share one E8M0
+ *     power-of-two scale.
+ *   - k is a parameter ("ds4-ssd" README, "Experimental Pro Support":
+ *     --moe-expert-topk changes the routed expert count); a shared,
+ *     always-on expert exists (same section: shared-down prefetch).
+ *   - the decode step (T = 1) and the speculative-verify batch of 1 + 4 draft
+ *     positions (10100.com ds4-ssd article, "运行模式" / DSpark mode:
+ *     --draft-verify 4) are the shapes the layer runs at; prefill runs in
+ *     chunks of up to 4K tokens ("ds4-ssd" README, "Validate").
+ *
+ * Readings where the pages are silent (the same readings as the CPU oracle):
+ *   logits = x W_r^T + b (bias used for selection and weights); softmax over
+ *   all E, top-k in descending logit order (ties -> lower expert index),
+ *   renormalised over the chosen k, no extra scaling; expert
+ *   o = W_down (silu(W_gate x) * (W_up x)); y = sum_j w_j o_j (slot order)
+ *   + o_shared, rounded to bf16 (RNE).
+ *
+ * Layouts (all row-major, all device memory unless stated otherwise):
+ *   x        [T, H]   bf16 bit patterns (uint16)
+ *   W_r      [E, H]   float32 router weights;  bias [E] float32 or NULL
+ *   topk_idx [T, k]   int32, descending logit order
+ *   topk_w   [T, k]   float32, rows sum to 1
+ *   counts   [E]      int32 tokens routed to each expert
+ *   offsets  [E + 1]  int32 exclusive scan of counts, offsets[E] = T*k
+ *   entries  [T*k]    int32 pair indices p = t*k + j sorted by expert, and by
+ *                     ascending token within one expert (stable)
+ *   experts  gate_q/up_q [n, I, H/2] u8, gate_s/up_s [n, I, H/32] u8,
+ *            down_q [n, H, I/2] u8, down_s [n, H, I/32] u8.  Byte b of a row
+ *            holds element 2b in its low nibble and 2b+1 in its high nibble;
+ *            scale byte q covers elements 32q..32q+31 of the row.
+ *   partial  [T*k + S*T, H] float32: row p = t*k + j is expert idx[t,j]'s
+ *            output for token t; rows T*k + t are the shared expert's (S = 1).
+ *   y        [T, H]   bf16 bit patterns
+ *
+ * Constraints (checked on the host before any launch): 1 <= T <= 65536,
+ * 32 <= H <= 16384 and H % 32 == 0, 32 <= I <= 16384 and I % 32 == 0,
+ * 1 <= E <= 1024, 1 <= k <= min(E, 16); every pointer 16-byte aligned.
+ * Violations return MOE_ERR_UNSUPPORTED_SHAPE or MOE_ERR_INVALID_ARG.
+ *
+ * Ownership and errors: the caller allocates every buffer; the library never
+ * allocates or frees device memory.  Calls are asynchronous on `stream`
+ * (a cudaStream_t; NULL = legacy default stream) and never synchronise the
+ * host.  A launch failure returns MOE_ERR_CUDA.  Faults found on the device
+ * (an expert index out of range, ...) are latched in the workspace and read
+ * with moe_get_error().  No C++ exception crosses this boundary.
+ *
+ * Workspace: `ws` is caller-owned device memory of at least
+ * moe_workspace_bytes(...) bytes, zeroed once by moe_workspace_init() before
+ * its first use.  Kernels leave its counters at zero, so one workspace serves
+ * any number of calls, including calls replayed from a CUDA graph, as long as
+ * calls sharing a workspace are ordered on one stream.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t moe_status_t;
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1)
+#define MOE_ERR_UNSUPPORTED_SHAPE (-2)
+#define MOE_ERR_WORKSPACE (-3)
+#define MOE_ERR_CUDA (-4)
+#define MOE_ERR_TIMEOUT (-5)
+#define MOE_ERR_DEVICE_DATA (-6)
+
+typedef struct moe_shape {
+  int32_t T; /* tokens in the batch */
+  int32_t H; /* hidden size (expert input / output width) */
+  int32_t I; /* expert intermediate size */
+  int32_t E; /* routed experts */
+  int32_t k; /* experts chosen per token */
+} moe_shape_t;
+
+/* Device pointers to n_experts MXFP4 experts in the layout above. */
+typedef struct moe_mxfp4_experts {
+  const uint8_t* gate_q;
+  const uint8_t* gate_s;
+  const uint8_t* up_q;
+  const uint8_t* up_s;
+  const uint8_t* down_q;
+  const uint8_t* down_s;
+  int32_t n_experts;
+} moe_mxfp4_experts_t;
+
+/* Expert FFN implementation.  GEMV: CUDA-core streaming kernels, exact bf16
+ * activations (decode / verify).  GEMM: tcgen05 block-scaled FP4 tensor-core
+ * kernels (prefill), which require MOE_ACT_MXFP4.  AUTO picks by batch size. */
+#define MOE_PATH_AUTO 0
+#define MOE_PATH_GEMV 1
+#define MOE_PATH_GEMM 2
+
+/* Activation precision of the expert projections.  EXACT: the bf16 token
+ * rows and the fp32 SwiGLU output enter the projections as they are (the
+ * pages' quality mode, "ds4-ssd" README, "Experimental Pro Support":
+ * --quality / --no-int8).  MXFP4: each projection input row is quantised to
+ * MXFP4 in 32-element blocks first (scale 2^(floor(log2 amax) - 2),
+ * round-to-nearest-even onto the E2M1 grid, saturating at +-6), as an
+ * accelerator path does. */
+#define MOE_ACT_EXACT 0
+#define MOE_ACT_MXFP4 1
+
+/* Bytes of workspace the calls below need for this shape (any of them).
+ * has_shared: 1 if a shared expert is passed.  Returns 0 for an unsupported
+ * shape, path or precision. */
+MOE_API size_t moe_workspace_bytes(moe_shape_t shape, int32_t path, int32_t precision,
+                           int32_t has_shared);
+
+/* Zero a workspace before its first use (asynchronous memset on stream). */
+MOE_API moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Router, softmax, top-k and renormalisation.
+ * logits[t,e] = sum_h x[t,h] W_r[e,h] + bias[e] in float32 (bias may be NULL);
+ * topk_idx/topk_w as described above.  logits_out [T, E] float32 may be NULL.
+ * Ties of equal float32 logits go to the lower expert index. */
+MOE_API moe_status_t moe_route_topk(const uint16_t* x, const float* w_router,
+                            const float* bias, moe_shape_t shape,
+                            float* logits_out, int32_t* topk_idx,
+                            float* topk_w, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/* Stable counting sort of the T*k (token, slot) pairs by expert: writes
+ * counts [E], offsets [E+1] and entries [T*k] (layouts above).  An index
+ * outside [0, E) latches MOE_ERR_DEVICE_DATA and the pair is dropped. */
+MOE_API moe_status_t moe_bucket(const int32_t* topk_idx, moe_shape_t shape,
+                        int32_t* counts, int32_t* offsets, int32_t* entries,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* Expert SwiGLU FFNs of the routed pairs (and of every token through the
+ * shared expert when `shared` is not NULL):
+ *   partial[p]      = W_down[e] (silu(W_gate[e] x_t) * (W_up[e] x_t))
+ *   for every p = t*k + j listed in entries with e the bucket's expert, and
+ *   partial[T*k+t]  = the same through the shared expert.
+ * `experts` and `shared` are host pointers to structs of device pointers;
+ * experts->n_experts must equal shape.E, shared->n_experts must be 1.
+ * Rows of pairs not listed in entries are left untouched. */
+MOE_API moe_status_t moe_expert_ffn_mxfp4(const moe_mxfp4_experts_t* experts,
+                                  const moe_mxfp4_experts_t* shared,
+                                  const uint16_t* x, const int32_t* offsets,
+                                  const int32_t* entries, moe_shape_t shape,
+                                  int32_t path, int32_t precision,
+                                  float* partial_out, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/* y[t] = bf16_rne( sum_{j<k} topk_w[t,j] * partial[t*k+j]
+ *                  + (has_shared ? partial[T*k+t] : 0) ), summed in that
+ * order in float32. */
+MOE_API moe_status_t moe_combine(const float* partial, const float* topk_w,
+                         moe_shape_t shape, int32_t has_shared, uint16_t* y,
+                         void* stream);
+
+/* The whole layer: route -> bucket -> expert FFNs -> combine, on `stream`.
+ * topk_idx_out [T,k] and topk_w_out [T,k] may be NULL (kept in ws then). */
+MOE_API moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router,
+                               const float* bias,
+                               const moe_mxfp4_experts_t* experts,
+                               const moe_mxfp4_experts_t* shared,
+                               moe_shape_t shape, int32_t path,
+                               int32_t precision, uint16_t* y,
+                               int32_t* topk_idx_out, float* topk_w_out,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/* Quantise rows [rows, K] float32 to MXFP4 (codes [rows, K/2], scales
+ * [rows, K/32]) with the MOE_ACT_MXFP4 rule above; K % 32 == 0. */
+MOE_API moe_status_t moe_act_quant_mxfp4(const float* in, int32_t rows, int32_t K,
+                                 uint8_t* q_out, uint8_t* s_out, void* stream);
+
+/* Decode MXFP4 rows (codes [rows, K/2], scales [rows, K/32]) to float32
+ * [rows, K] with the same in-register decode the FFN kernels use (E2M1 value
+ * times 2^(scale-127); scale byte 255 gives NaN).  For tests and tools. */
+MOE_API moe_status_t moe_decode_mxfp4(const uint8_t* q, const uint8_t* s, int32_t rows,
+                              int32_t K, float* out, void* stream);
+
+/* Synchronise `stream`, return the first device-side error latched in ws
+ * since the last call (MOE_OK if none) and clear it. */
+MOE_API moe_status_t moe_get_error(void* ws, void* stream);
+
+/* Static description of a status code. */
+MOE_API const char* moe_status_string(moe_status_t status);
+
+/* Library version, e.g. "0.1.0". */
+MOE_API const char* moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,476 @@
+// Grouped GEMV over the activated MXFP4 experts (decode / verify batches).
+//
+// Only the experts some token chose are read (ainews.cool "antirez ds4
+// DeepSeek Metal inference", 技术深度解析: block-sparse matmul that loads only
+// activated experts' weights; "ds4-ssd" README, "Run SSD Sidecar Mode":
+// MXFP4 routed experts).  Each projection row is dequantised in registers:
+// a lane loads one 16-byte chunk = one 32-element MX block (so one E8M0
+// scale per lane per row), converts the E2M1 pairs with the sm_100a
+// cvt.rn.f16x2.e2m1x2 instruction, multiplies by the token rows held in
+// registers and accumulates in float32; the block's power-of-two scale is
+// applied once to the block sum.
+//
+// Work split ("virtual experts"): v < nA is the v-th activated routed expert
+// (ascending id, from the bucket's plan); v == nA is the shared expert when
+// present.  A projection's rows of all virtual experts form one list of
+// nV * ROWS units; every CTA of the persistent grid takes an equal contiguous
+// range of it, so HBM traffic is spread evenly over the SMs whatever the
+// routing.  Phase 0 (gate/up): ROWS = I, each unit is gate row i and up row i,
+// the epilogue writes h = silu(g) * u.  Phase 1 (down): ROWS = H, each unit is
+// one output row d, the epilogue writes the expert output into `partial`.
+//
+// Inside a CTA (4 warps) the K dimension of a row is split over KS warps
+// (KS = 1, 2 or 4, 32*KS lanes cover the row's blocks); the 4/KS warp groups
+// work on different units.  A warp accumulates UG units x NPROJ projections x
+// RC tokens, then one butterfly "transpose" reduction over its 32 lanes
+// leaves one finished value per lane (31 shuffles for 32 values instead of
+// 5 per value); the KS warps' partial sums are added in shared memory.
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr int kPiece = 64;  // units per epilogue piece
+
+// Arithmetic policies for one 32-element block dot product.
+enum Policy : int {
+  kMixed = 0,  // x in f16; fma.rn.f32.f16 (exact f16 products, f32 accumulate)
+  kF32x2 = 1,  // x in f32; weights widened to f32; packed fma.rn.f32x2
+};
+
+template <int POL>
+struct XReg;
+template <>
+struct XReg<kMixed> {
+  uint32_t v[16];  // f16x2 pairs (x[2j], x[2j+1])
+};
+template <>
+struct XReg<kF32x2> {
+  float2 v[16];
+};
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  unsigned long long ra, rb, rc, rd;
+  ra = (static_cast<unsigned long long>(__float_as_uint(a.y)) << 32) | __float_as_uint(a.x);
+  rb = (static_cast<unsigned long long>(__float_as_uint(b.y)) << 32) | __float_as_uint(b.x);
+  rc = (static_cast<unsigned long long>(__float_as_uint(c.y)) << 32) | __float_as_uint(c.x);
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
+  return make_float2(__uint_as_float(uint32_t(rd)), __uint_as_float(uint32_t(rd >> 32)));
+}
+
+// 32 float values of a block -> the policy's register form.  With act_mxfp4
+// the block is first quantised to MXFP4 and dequantised (OCP MX v1.0 scale
+// 2^(floor(log2 amax) - 2), RNE onto E2M1, saturating), which is exactly the
+// value an MXFP4 activation operand carries.
+template <int POL>
+__device__ __forceinline__ void pack_block(float (&f)[32], bool act_mxfp4, XReg<POL>& out) {
+  if (act_mxfp4) {
+    float amax = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(f[j]));
+    const int X = mx_scale_exponent(amax);
+    const float inv = exp2i(-X > 127 ? 127 : -X);
+    const float sc = exp2i(X);
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) {
+      uint32_t byte4 = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        byte4 |= f32x2_to_e2m1x2(f[j + 2 * b] * inv, f[j + 2 * b + 1] * inv) << (8 * b);
+      uint32_t h2[4];
+      e2m1x8_to_f16x2(byte4, h2);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const float2 d = f16x2_to_f32x2(h2[b]);
+        f[j + 2 * b] = d.x * sc;
+        f[j + 2 * b + 1] = d.y * sc;
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    if constexpr (POL == kMixed) out.v[j] = f32x2_to_f16x2(f[2 * j], f[2 * j + 1]);
+    else out.v[j] = make_float2(f[2 * j], f[2 * j + 1]);
+  }
+}
+
+__device__ __forceinline__ void load_block_bf16(const uint16_t* row, int b, float (&f)[32]) {
+  const uint4* p = reinterpret_cast<const uint4*>(row + size_t(b) * 32);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 v = __ldg(p + q);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      f[8 * q + 2 * j] = bf16_bits_to_f32(w[j] & 0xffffu);
+      f[8 * q + 2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+    }
+  }
+}
+
+__device__ __forceinline__ void load_block_f32(const float* row, int b, float (&f)[32]) {
+  const float4* p = reinterpret_cast<const float4*>(row + size_t(b) * 32);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 v = __ldcg(p + q);  // written by the previous kernel: bypass L1
+    f[4 * q] = v.x;
+    f[4 * q + 1] = v.y;
+    f[4 * q + 2] = v.z;
+    f[4 * q + 3] = v.w;
+  }
+}
+
+template <int POL>
+struct BlockW {
+  uint32_t h[16];  // f16x2 weight pairs
+};
+
+__device__ __forceinline__ void decode_codes(const uint4& c, uint32_t (&h)[16]) {
+  uint32_t t[4];
+  e2m1x8_to_f16x2(c.x, t);
+  h[0] = t[0]; h[1] = t[1]; h[2] = t[2]; h[3] = t[3];
+  e2m1x8_to_f16x2(c.y, t);
+  h[4] = t[0]; h[5] = t[1]; h[6] = t[2]; h[7] = t[3];
+  e2m1x8_to_f16x2(c.z, t);
+  h[8] = t[0]; h[9] = t[1]; h[10] = t[2]; h[11] = t[3];
+  e2m1x8_to_f16x2(c.w, t);
+  h[12] = t[0]; h[13] = t[1]; h[14] = t[2]; h[15] = t[3];
+}
+
+template <int POL>
+__device__ __forceinline__ float block_dot(const uint32_t (&w)[16], const XReg<POL>& x) {
+  if constexpr (POL == kMixed) {
+    float a0 = 0.f, a1 = 0.f;  // two chains for latency
+#pragma unroll
+    for (int j = 0; j < 16; j += 2) {
+      a0 = fma2_f16_f32(w[j], x.v[j], a0);
+      a1 = fma2_f16_f32(w[j + 1], x.v[j + 1], a1);
+    }
+    return a0 + a1;
+  } else {
+    float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) a = ffma2(f16x2_to_f32x2(w[j]), x.v[j], a);
+    return a.x + a.y;
+  }
+}
+
+// Butterfly reduce-scatter of NVAL per-lane values over the warp: afterwards
+// every lane holds the warp total of value index (lane & (NVAL - 1)).
+template <int NVAL>
+__device__ __forceinline__ float transpose_reduce(float (&v)[NVAL], int lane) {
+#pragma unroll
+  for (int m = NVAL / 2; m >= 1; m >>= 1) {
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int i = 0; i < m; ++i) {
+      const float keep = upper ? v[i + m] : v[i];
+      const float send = upper ? v[i] : v[i + m];
+      v[i] = keep + __shfl_xor_sync(kFull, send, m);
+    }
+  }
+#pragma unroll
+  for (int m = NVAL; m < 32; m <<= 1) v[0] += __shfl_xor_sync(kFull, v[0], m);
+  return v[0];
+}
+
+struct VExpert {
+  const uint8_t* q[2];
+  const uint8_t* s[2];
+  const int32_t* rows;  // pair indices of the bucket, or nullptr for the shared expert
+  int R;                // tokens
+};
+
+__device__ __forceinline__ VExpert vexpert(const FfnArgs& a, int phase, int v, int nA) {
+  VExpert ve;
+  const int K = phase == 0 ? a.H : a.I;
+  const int ROWS = phase == 0 ? a.I : a.H;
+  const size_t mat = size_t(ROWS) * (K / 2), smat = size_t(ROWS) * (K / 32);
+  if (v < nA) {
+    const int e = a.plan[1 + v];
+    const int beg = a.offsets[e], end = a.offsets[e + 1];
+    ve.rows = a.entries + beg;
+    ve.R = end - beg;
+    if (phase == 0) {
+      ve.q[0] = a.ex.gq + e * mat; ve.s[0] = a.ex.gs + e * smat;
+      ve.q[1] = a.ex.uq + e * mat; ve.s[1] = a.ex.us + e * smat;
+    } else {
+      ve.q[0] = a.ex.dq + e * mat; ve.s[0] = a.ex.ds + e * smat;
+      ve.q[1] = nullptr; ve.s[1] = nullptr;
+    }
+  } else {
+    ve.rows = nullptr;
+    ve.R = a.T;
+    if (phase == 0) {
+      ve.q[0] = a.sh.gq; ve.s[0] = a.sh.gs;
+      ve.q[1] = a.sh.uq; ve.s[1] = a.sh.us;
+    } else {
+      ve.q[0] = a.sh.dq; ve.s[0] = a.sh.ds;
+      ve.q[1] = nullptr; ve.s[1] = nullptr;
+    }
+  }
+  return ve;
+}
+
+// Output row (pair index, or T*k + t for the shared expert) of bucket row r.
+__device__ __forceinline__ int out_row(const FfnArgs& a, const VExpert& ve, int r) {
+  return ve.rows ? ve.rows[r] : a.T * a.k + r;
+}
+__device__ __forceinline__ int token_of(const FfnArgs& a, const VExpert& ve, int r) {
+  return ve.rows ? ve.rows[r] / a.k : r;
+}
+
+// One virtual expert, units [r0, r1), tokens [t0, t0 + nt) of its bucket.
+template <int PHASE, int POL, int RC, int BPL>
+__device__ void run_span(const FfnArgs& a, const VExpert& ve, int r0, int r1, int t0, int nt,
+                         int KS, float* part) {
+  constexpr int NPROJ = PHASE == 0 ? 2 : 1;
+  // units per group: at most 16 code loads in flight per lane, at most 32
+  // accumulators (the butterfly reduction works on a power of two <= 32)
+  constexpr int UG_LOAD = 16 / (NPROJ * BPL) > 0 ? 16 / (NPROJ * BPL) : 1;
+  constexpr int UG_ACC = 32 / (NPROJ * RC) > 0 ? 32 / (NPROJ * RC) : 1;
+  constexpr int UG = UG_LOAD < UG_ACC ? UG_LOAD : UG_ACC;
+  constexpr int NVAL = UG * NPROJ * RC;
+  static_assert((NVAL & (NVAL - 1)) == 0 && NVAL <= 32, "NVAL must be a power of two <= 32");
+  const int K = PHASE == 0 ? a.H : a.I;
+  const int ROWS = PHASE == 0 ? a.I : a.H;
+  const int nb = K / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int NG = kWarps / KS;
+  const int grp = warp / KS;
+  const int gl = (warp % KS) * 32 + lane;  // lane index within the K group
+  const int lstride = 32 * KS;
+
+  // token rows -> registers
+  XReg<POL> xr[BPL][RC];
+#pragma unroll
+  for (int m = 0; m < BPL; ++m) {
+    const int b = gl + m * lstride;
+#pragma unroll
+    for (int t = 0; t < RC; ++t) {
+      float f[32];
+      if (t < nt && b < nb) {
+        const int r = t0 + t;
+        if constexpr (PHASE == 0) {
+          load_block_bf16(a.x + size_t(token_of(a, ve, r)) * a.H, b, f);
+        } else {
+          load_block_f32(a.h + size_t(out_row(a, ve, r)) * a.I, b, f);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) f[j] = 0.f;
+      }
+      pack_block<POL>(f, a.act_mxfp4 != 0, xr[m][t]);
+    }
+  }
+
+  const size_t rowq = size_t(K) / 2;
+  for (int p0 = r0; p0 < r1; p0 += kPiece) {
+    const int np = min(kPiece, r1 - p0);
+    const int gbeg = (grp * np) / NG, gend = ((grp + 1) * np) / NG;
+    for (int g = gbeg; g < gend; g += UG) {
+      float acc[NVAL];
+#pragma unroll
+      for (int i = 0; i < NVAL; ++i) acc[i] = 0.f;
+      uint4 cq[UG][NPROJ][BPL];
+      uint32_t cs[UG][NPROJ][BPL];
+#pragma unroll
+      for (int u = 0; u < UG; ++u) {
+        const int row = p0 + g + u;
+        const bool uv = (g + u) < gend;
+#pragma unroll
+        for (int pj = 0; pj < NPROJ; ++pj) {
+#pragma unroll
+          for (int m = 0; m < BPL; ++m) {
+            const int b = gl + m * lstride;
+            if (uv && b < nb) {
+              cq[u][pj][m] = ldg_stream(ve.q[pj] + size_t(row) * rowq + size_t(b) * 16);
+              cs[u][pj][m] = ldg_u8(ve.s[pj] + size_t(row) * nb + b);
+            } else {
+              cq[u][pj][m] = make_uint4(0, 0, 0, 0);
+              cs[u][pj][m] = 127u;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < UG; ++u) {
+#pragma unroll
+        for (int pj = 0; pj < NPROJ; ++pj) {
+#pragma unroll
+          for (int m = 0; m < BPL; ++m) {
+            uint32_t w[16];
+            decode_codes(cq[u][pj][m], w);
+            const float sc = e8m0_to_f32(cs[u][pj][m]);
+#pragma unroll
+            for (int t = 0; t < RC; ++t) {
+              const float bs = block_dot<POL>(w, xr[m][t]);
+              float& dst = acc[(u * NPROJ + pj) * RC + t];
+              dst = fmaf(sc, bs, dst);
+            }
+          }
+        }
+      }
+      const float tot = transpose_reduce<NVAL>(acc, lane);
+      if (lane < NVAL) {
+        const int t = lane % RC;
+        const int pj = (lane / RC) % NPROJ;
+        const int u = lane / (RC * NPROJ);
+        if (g + u < gend) part[((warp * kPiece + g + u) * NPROJ + pj) * RC + t] = tot;
+      }
+    }
+    __syncthreads();
+    // epilogue: add the KS warps' partial sums of each unit
+    for (int q = threadIdx.x; q < np * nt; q += kThreads) {
+      const int uix = q % np, t = q / np;
+      int owner = 0;
+      for (int gi = 1; gi < NG; ++gi)
+        if ((gi * np) / NG <= uix) owner = gi;
+      float s0 = 0.f, s1 = 0.f;
+      for (int w = owner * KS; w < owner * KS + KS; ++w) {
+        s0 += part[((w * kPiece + uix) * NPROJ + 0) * RC + t];
+        if constexpr (NPROJ == 2) s1 += part[((w * kPiece + uix) * NPROJ + 1) * RC + t];
+      }
+      const int orow = out_row(a, ve, t0 + t);
+      if constexpr (PHASE == 0) {
+        const float hval = s0 / (1.f + expf(-s0)) * s1;  // silu(g) * u
+        a.h[size_t(orow) * a.I + p0 + uix] = hval;
+      } else {
+        a.partial[size_t(orow) * a.H + p0 + uix] = s0;
+      }
+    }
+    __syncthreads();
+  }
+  (void)ROWS;
+}
+
+template <int PHASE, int POL, int RCMAX, int BPL>
+__global__ void __launch_bounds__(kThreads) k_ffn_gemv(FfnArgs a, int KS) {
+  __shared__ float part[kWarps * kPiece * (PHASE == 0 ? 2 : 1) * RCMAX];
+  pdl_wait();
+  pdl_trigger();
+  const int nA = a.plan[0];
+  const int nV = nA + (a.has_shared ? 1 : 0);
+  const int ROWS = PHASE == 0 ? a.I : a.H;
+  const long long U = (long long)nV * ROWS;
+  const long long ub = U * blockIdx.x / gridDim.x;
+  const long long ue = U * (blockIdx.x + 1) / gridDim.x;
+  long long u = ub;
+  while (u < ue) {
+    const int v = int(u / ROWS);
+    const int r0 = int(u % ROWS);
+    const int r1 = int(min((long long)ROWS, r0 + (ue - u)));
+    const VExpert ve = vexpert(a, PHASE, v, nA);
+    for (int t0 = 0; t0 < ve.R; t0 += RCMAX) {
+      const int nt = min(RCMAX, ve.R - t0);
+      // smallest register tile holding the chunk
+      if (RCMAX >= 4 && nt > 2) {
+        run_span<PHASE, POL, (RCMAX >= 4 ? 4 : RCMAX), BPL>(a, ve, r0, r1, t0, nt, KS, part);
+      } else if (RCMAX >= 2 && nt == 2) {
+        run_span<PHASE, POL, (RCMAX >= 2 ? 2 : RCMAX), BPL>(a, ve, r0, r1, t0, nt, KS, part);
+      } else {
+        run_span<PHASE, POL, 1, BPL>(a, ve, r0, r1, t0, nt, KS, part);
+      }
+    }
+    u += r1 - r0;
+  }
+}
+
+template <int PHASE, int POL>
+cudaError_t launch_phase(const FfnArgs& a, int grid, cudaStream_t st) {
+  const int K = PHASE == 0 ? a.H : a.I;
+  const int nb = K / 32;
+  int KS, BPL;
+  if (nb <= 32) { KS = 1; BPL = 1; }
+  else if (nb <= 64) { KS = 2; BPL = 1; }
+  else if (nb <= 128) { KS = 4; BPL = 1; }
+  else if (nb <= 256) { KS = 4; BPL = 2; }
+  else { KS = 4; BPL = 4; }
+  // register tile of tokens: at most 4 per pass, fewer for wide rows
+  const int rcmax_cap = BPL == 1 ? 4 : (BPL == 2 ? 2 : 1);
+  int RCMAX = a.T >= 4 ? 4 : (a.T >= 2 ? 2 : 1);
+  if (RCMAX > rcmax_cap) RCMAX = rcmax_cap;
+  const dim3 g(grid), b(kThreads);
+#define MOE_GEMV_CASE(RCM, B)                                                          \
+  if (RCMAX == RCM && BPL == B) return launch_pdl(k_ffn_gemv<PHASE, POL, RCM, B>, g, b, 0, st, a, KS);
+  MOE_GEMV_CASE(1, 1)
+  MOE_GEMV_CASE(2, 1)
+  MOE_GEMV_CASE(4, 1)
+  MOE_GEMV_CASE(1, 2)
+  MOE_GEMV_CASE(2, 2)
+  MOE_GEMV_CASE(1, 4)
+#undef MOE_GEMV_CASE
+  return cudaErrorInvalidValue;
+}
+
+__global__ void __launch_bounds__(256) k_combine(const float* partial, const float* w, int T,
+                                                 int H, int k, int has_shared, uint16_t* y) {
+  pdl_wait();
+  pdl_trigger();
+  const int per_row = H / 4;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)T * per_row) return;
+  const int t = int(i / per_row), c = int(i % per_row) * 4;
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < k; ++j) {
+    const float wj = __ldcg(w + size_t(t) * k + j);
+    const float4 p = __ldcg(reinterpret_cast<const float4*>(partial + (size_t(t) * k + j) * H + c));
+    s.x = fmaf(wj, p.x, s.x);
+    s.y = fmaf(wj, p.y, s.y);
+    s.z = fmaf(wj, p.z, s.z);
+    s.w = fmaf(wj, p.w, s.w);
+  }
+  if (has_shared) {
+    const float4 p =
+        __ldcg(reinterpret_cast<const float4*>(partial + (size_t(T) * k + t) * H + c));
+    s.x += p.x;
+    s.y += p.y;
+    s.z += p.z;
+    s.w += p.w;
+  }
+  __nv_bfloat162 lo = __floats2bfloat162_rn(s.x, s.y), hi = __floats2bfloat162_rn(s.z, s.w);
+  uint2 out;
+  out.x = *reinterpret_cast<uint32_t*>(&lo);
+  out.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(y + size_t(t) * H + c) = out;
+}
+
+}  // namespace
+
+#ifndef MOE_GEMV_POLICY
+#define MOE_GEMV_POLICY 0
+#endif
+
+int gemv_grid(int phase) {
+  static int occ[2] = {0, 0};
+  const DeviceInfo di = device_info();
+  if (occ[phase] == 0) {
+    int o = 0;
+    if (phase == 0)
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_ffn_gemv<0, MOE_GEMV_POLICY, 4, 1>,
+                                                    kThreads, 0);
+    else
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_ffn_gemv<1, MOE_GEMV_POLICY, 4, 1>,
+                                                    kThreads, 0);
+    occ[phase] = o > 0 ? o : 1;
+  }
+  return di.sm_count * occ[phase];
+}
+
+cudaError_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t st) {
+  cudaError_t e = launch_phase<0, MOE_GEMV_POLICY>(a, gemv_grid(0), st);
+  if (e != cudaSuccess) return e;
+  return launch_phase<1, MOE_GEMV_POLICY>(a, gemv_grid(1), st);
+}
+
+cudaError_t launch_combine(const float* partial, const float* w, int T, int H, int k,
+                           int has_shared, uint16_t* y, cudaStream_t st) {
+  const long long n = (long long)T * (H / 4);
+  const int blocks = int((n + 255) / 256);
+  return launch_pdl(k_combine, dim3(blocks), dim3(256), 0, st, partial, w, T, H, k, has_shared,
+                    y);
+}
+
+}  // namespace moe

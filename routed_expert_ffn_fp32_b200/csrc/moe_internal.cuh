@@ -1,0 +1,260 @@
+// Internal declarations of the MXFP4 routed-MoE library (sm_100a).
+//
+// Device helpers shared by the kernels, the workspace layout, and the launch
+// functions each kernel file provides to the C-ABI layer (moe_abi.cu).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 16;
+constexpr unsigned kFull = 0xffffffffu;
+
+// ---------------------------------------------------------------------------
+// Workspace layout.  Every region starts on a 256-byte boundary.
+// ---------------------------------------------------------------------------
+struct WsLayout {
+  size_t err;       // int32[16]: [0] status, [1] detail
+  size_t counters;  // uint32[16]: arrival counters, zero between calls
+  size_t logits;    // f32 [T, E]
+  size_t idx;       // i32 [T, k]
+  size_t w;         // f32 [T, k]
+  size_t counts;    // i32 [E]
+  size_t offsets;   // i32 [E + 1]
+  size_t entries;   // i32 [T * k]
+  size_t plan;      // i32 [E + 2]: [0] active experts, [1..] their ids (ascending)
+  size_t h;         // f32 [T*k + S*T, I]   SwiGLU output rows (by pair index)
+  size_t partial;   // f32 [T*k + S*T, H]   expert output rows (by pair index)
+  size_t aq;        // u8  [T*k + S*T, max(H,I)/2]  MXFP4 activation codes (GEMM path)
+  size_t as;        // u8  [T*k + S*T, max(H,I)/32] MXFP4 activation scales (GEMM path)
+  size_t total;
+};
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+__host__ __device__ inline size_t align_up16(size_t v) { return (v + 15) & ~size_t(15); }
+
+inline WsLayout ws_layout(const moe_shape_t& s, int has_shared, int gemm) {
+  WsLayout L{};
+  const size_t T = s.T, H = s.H, I = s.I, E = s.E, k = s.k;
+  const size_t rows = T * k + (has_shared ? T : 0);
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
+  L.err = take(64);
+  L.counters = take(64);
+  L.logits = take(T * E * 4);
+  L.idx = take(T * k * 4);
+  L.w = take(T * k * 4);
+  L.counts = take(E * 4);
+  L.offsets = take((E + 1) * 4);
+  L.entries = take(T * k * 4);
+  L.plan = take((E + 2) * 4);
+  L.h = take(rows * I * 4);
+  L.partial = take(rows * H * 4);
+  const size_t KM = H > I ? H : I;
+  L.aq = gemm ? take(rows * KM / 2) : o;
+  L.as = gemm ? take(rows * KM / 32) : o;
+  L.total = o;
+  return L;
+}
+
+// ---------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void latch_error(int* err, int code, int detail) {
+  if (atomicCAS(err, 0, code) == 0) atomicExch(err + 1, detail);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) {
+  return __uint_as_float(b << 16);
+}
+
+// E8M0 scale byte -> 2^(s-127) as float32.  s = 0 is the subnormal 2^-127,
+// s = 255 is NaN (OCP MX v1.0, E8M0).
+__device__ __forceinline__ float e8m0_to_f32(uint32_t s) {
+  uint32_t bits = s << 23;
+  bits = (s == 0u) ? 0x00400000u : bits;
+  bits = (s == 255u) ? 0x7fc00000u : bits;
+  return __uint_as_float(bits);
+}
+
+// Four bytes of E2M1 pairs -> four f16x2 registers (hardware cvt, sm_100a).
+// Byte j (bits 8j..8j+7) holds elements 2j (low nibble) and 2j+1 (high
+// nibble); out[j] holds them as (low half, high half).
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&out)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(out[0]), "=r"(out[1]), "=r"(out[2]), "=r"(out[3])
+      : "r"(w));
+}
+
+// acc += w.lo * x.lo + w.hi * x.hi with f16 inputs and an f32 accumulator:
+// each product is exact and is added to acc with one f32 rounding.
+__device__ __forceinline__ float fma2_f16_f32(uint32_t w2, uint32_t x2, float acc) {
+  asm("{\n\t.reg .f16 wl, wh, xl, xh;\n\t"
+      "mov.b32 {wl, wh}, %1;\n\t"
+      "mov.b32 {xl, xh}, %2;\n\t"
+      "fma.rn.f32.f16 %0, wl, xl, %0;\n\t"
+      "fma.rn.f32.f16 %0, wh, xh, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(w2), "r"(x2));
+  return acc;
+}
+
+__device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t v) {
+  __half2 h = *reinterpret_cast<__half2*>(&v);
+  return __half22float2(h);
+}
+
+__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Two floats -> one byte of two E2M1 codes (lo -> low nibble), RNE, saturating.
+__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 r;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 r, %2, %1;\n\t"
+      "cvt.u32.u8 %0, r;\n\t}"
+      : "=r"(out)
+      : "f"(lo), "f"(hi));
+  return out;
+}
+
+// Streaming 16-byte load that does not allocate in L1 (weights are read once).
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t ldg_u8(const uint8_t* p) {
+  return static_cast<uint32_t>(__ldg(p));
+}
+
+// Programmatic dependent launch: wait for the preceding kernel's memory, then
+// let the next kernel's blocks be scheduled.  Both are no-ops without PDL.
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" :::);
+}
+
+// MXFP4 scale exponent of a block from its largest magnitude (OCP MX v1.0:
+// X = floor(log2 amax) - emax(E2M1) with emax = 2, clamped to [-127, 127];
+// amax = 0 gives -127).
+__device__ __forceinline__ int mx_scale_exponent(float amax) {
+  const uint32_t bits = __float_as_uint(amax) & 0x7fffffffu;
+  const int ef = int(bits >> 23);  // biased exponent; 0 for zero and subnormals
+  if (ef == 0) return -127;        // floor(log2 amax) - 2 < -127: clamps
+  const int X = ef - 127 - 2;
+  return X > 127 ? 127 : X;
+}
+
+// 2^e as a float for e in [-127, 127] (e = -127 is the subnormal 2^-127).
+__device__ __forceinline__ float exp2i(int e) {
+  return e >= -126 ? __uint_as_float(uint32_t(e + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// ---------------------------------------------------------------------------
+// Kernel argument blocks
+// ---------------------------------------------------------------------------
+struct ExpertPtrs {
+  const uint8_t* gq;
+  const uint8_t* gs;
+  const uint8_t* uq;
+  const uint8_t* us;
+  const uint8_t* dq;
+  const uint8_t* ds;
+};
+
+struct RouteArgs {
+  const uint16_t* x;
+  const float* w_router;
+  const float* bias;
+  float* logits;
+  int32_t* idx;
+  float* w;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* entries;
+  int32_t* plan;
+  uint32_t* counter;
+  int* err;
+  int T, H, E, k;
+};
+
+struct FfnArgs {
+  ExpertPtrs ex;
+  ExpertPtrs sh;  // shared expert (n = 1) when has_shared
+  const uint16_t* x;
+  const int32_t* offsets;
+  const int32_t* entries;
+  const int32_t* plan;
+  const float* topk_w;  // down kernel with combine
+  float* h;             // [rows, I]
+  float* partial;       // [rows, H]
+  uint16_t* y;          // combine output or nullptr
+  int* err;
+  int T, H, I, E, k;
+  int has_shared;
+  int act_mxfp4;
+};
+
+// ---------------------------------------------------------------------------
+// Launchers (return cudaError_t of the launch)
+// ---------------------------------------------------------------------------
+struct DeviceInfo {
+  int sm_count;
+  int max_smem_optin;
+};
+DeviceInfo device_info();
+
+cudaError_t launch_route_logits(const RouteArgs& a, bool fuse_tail, cudaStream_t st);
+size_t route_fused_smem(int T, int H, int E, int k);
+cudaError_t launch_topk(const RouteArgs& a, cudaStream_t st);
+cudaError_t launch_bucket(const RouteArgs& a, cudaStream_t st);
+cudaError_t launch_plan(const RouteArgs& a, cudaStream_t st);
+
+cudaError_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t st);
+cudaError_t launch_combine(const float* partial, const float* w, int T, int H, int k,
+                           int has_shared, uint16_t* y, cudaStream_t st);
+cudaError_t launch_act_quant(const float* in, int rows, int K, uint8_t* q, uint8_t* s,
+                             cudaStream_t st);
+cudaError_t launch_decode(const uint8_t* q, const uint8_t* s, int rows, int K, float* out,
+                          cudaStream_t st);
+
+// Launch helper: every kernel goes out with programmatic stream serialisation
+// so its blocks can be scheduled while the previous kernel drains; each
+// kernel calls pdl_wait() before its first global memory access.
+template <typename Kernel, typename... Args>
+cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+}  // namespace moe

@@ -1,0 +1,427 @@
+// Router logits, softmax / top-k / renormalise, and the stable bucket of
+// (token, slot) pairs by expert.
+//
+// The pages only say that a token activates a few experts (ainews.cool
+// "antirez ds4 DeepSeek Metal inference", 技术深度解析: top-k routing over
+// fine-grained experts) and that k is a run-time knob ("ds4-ssd" README,
+// "Experimental Pro Support": --moe-expert-topk).  Formulas used here:
+//   logits[t,e] = sum_h x[t,h] W_r[e,h] + b[e]           (float32)
+//   idx[t,:]    = the k largest logits, descending, ties to the lower index
+//   w[t,j]      = exp(l_j - l_0) / sum_{j'<k} exp(l_j' - l_0)
+// which equals softmax over all E followed by renormalisation over the k.
+//
+// Kernels
+//   k_route_logits<TT>: one CTA per (2 experts, TT tokens).  Eight warps:
+//     warp w takes expert (w / 4) of the pair and the w % 4 quarter of H; each
+//     lane streams float4 router rows and keeps TT float32 partial sums.  The
+//     bf16 token rows sit in shared memory.  Every product meets at most
+//     H/128 + 9 roundings (lane chain, 5 shuffle levels, 3 quarter sums, the
+//     bias), the bound the parity tests use for near-ties.
+//     With fuse_tail the CTA that finishes last (arrival counter in the
+//     workspace, reset to zero by that CTA) runs top-k and the bucket for the
+//     whole batch, so a decode step routes in one launch.
+//   k_topk: one warp per token.
+//   k_bucket: one CTA; counts by shared-memory atomics, exclusive scan, then a
+//     stable placement of each 1024-pair chunk: ranks among equal experts come
+//     from __match_any_sync inside a warp plus per-warp counts of earlier warps.
+#include <float.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kRouteThreads = 256;
+constexpr int kBucketThreads = 1024;
+
+// ----------------------------------------------------------------- top-k ---
+template <int NV>
+__device__ void topk_warp(const float* row, int E, int k, int32_t* idx_out, float* w_out,
+                          int32_t* idx_smem) {
+  const int lane = threadIdx.x & 31;
+  float v[NV];
+  uint32_t removed = 0;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int e = lane + 32 * i;
+    float val = -FLT_MAX;
+    if (e < E) {
+      val = __ldcg(row + e);
+      if (val != val) val = -INFINITY;  // NaN ranks lowest
+    } else {
+      removed |= 1u << i;
+    }
+    v[i] = val;
+  }
+  float my_v = -INFINITY;
+  int my_i = 0;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int e = lane + 32 * i;
+      const bool live = !((removed >> i) & 1u);
+      if (live && (v[i] > bv || (v[i] == bv && e < bi))) {
+        bv = v[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const float ov = __shfl_xor_sync(kFull, bv, off);
+      const int oi = __shfl_xor_sync(kFull, bi, off);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if ((bi & 31) == lane) removed |= 1u << (bi >> 5);
+    if (lane == j) {
+      my_v = bv;
+      my_i = bi;
+    }
+  }
+  const float vmax = __shfl_sync(kFull, my_v, 0);
+  float p = (lane < k) ? expf(my_v - vmax) : 0.f;
+  float sum = p;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
+  if (lane < k) {
+    idx_out[lane] = my_i;
+    w_out[lane] = p / sum;
+    if (idx_smem) idx_smem[lane] = my_i;
+  }
+}
+
+template <typename F>
+__device__ void dispatch_nv(int E, F&& f) {
+  if (E <= 32) f.template operator()<1>();
+  else if (E <= 64) f.template operator()<2>();
+  else if (E <= 128) f.template operator()<4>();
+  else if (E <= 256) f.template operator()<8>();
+  else if (E <= 512) f.template operator()<16>();
+  else f.template operator()<32>();
+}
+
+__device__ void topk_block(const RouteArgs& a, int32_t* idx_smem) {
+  const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int t = warp; t < a.T; t += nwarps) {
+    const float* row = a.logits + size_t(t) * a.E;
+    int32_t* is = idx_smem ? idx_smem + t * a.k : nullptr;
+    dispatch_nv(a.E, [&]<int NV>() {
+      topk_warp<NV>(row, a.E, a.k, a.idx + size_t(t) * a.k, a.w + size_t(t) * a.k, is);
+    });
+  }
+}
+
+// ---------------------------------------------------------------- bucket ---
+struct BucketSmem {
+  int* cnt;       // [E]
+  int* cur;       // [E]
+  int* wsum;      // [2 * 33]
+  uint8_t* hist;  // [nwarps * E]
+};
+
+__device__ __forceinline__ BucketSmem bucket_smem(void* base, int E, int nwarps) {
+  BucketSmem s;
+  s.cnt = reinterpret_cast<int*>(base);
+  s.cur = s.cnt + E;
+  s.wsum = s.cur + E;
+  s.hist = reinterpret_cast<uint8_t*>(s.wsum + 2 * 33);
+  (void)nwarps;
+  return s;
+}
+
+inline size_t bucket_smem_bytes(int E, int nthreads) {
+  return size_t(E) * 8 + 2 * 33 * 4 + size_t(nthreads / 32) * E;
+}
+
+// Block-wide exclusive scan of per-thread (a, b) pairs; returns the exclusive
+// prefix of each and writes the totals.
+__device__ __forceinline__ void block_scan2(int a, int b, int& ea, int& eb, int& ta, int& tb,
+                                            int* wsum) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  int ia = a, ib = b;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int ua = __shfl_up_sync(kFull, ia, off), ub = __shfl_up_sync(kFull, ib, off);
+    if (lane >= off) {
+      ia += ua;
+      ib += ub;
+    }
+  }
+  if (lane == 31) {
+    wsum[warp] = ia;
+    wsum[33 + warp] = ib;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int va = lane < nwarps ? wsum[lane] : 0, vb = lane < nwarps ? wsum[33 + lane] : 0;
+    int sa = va, sb = vb;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int ua = __shfl_up_sync(kFull, sa, off), ub = __shfl_up_sync(kFull, sb, off);
+      if (lane >= off) {
+        sa += ua;
+        sb += ub;
+      }
+    }
+    if (lane < nwarps) {
+      wsum[lane] = sa - va;  // exclusive warp prefix
+      wsum[33 + lane] = sb - vb;
+    }
+    if (lane == 31) {
+      wsum[32] = sa;
+      wsum[65] = sb;
+    }
+  }
+  __syncthreads();
+  ea = wsum[warp] + ia - a;
+  eb = wsum[33 + warp] + ib - b;
+  ta = wsum[32];
+  tb = wsum[65];
+  __syncthreads();
+}
+
+// counts[] -> offsets[] / plan[] (active experts ascending); also primes cur[].
+__device__ void offsets_and_plan(const int* cnt, int E, int32_t* counts, int32_t* offsets,
+                                 int32_t* plan, int* cur, int* wsum) {
+  const int nthreads = blockDim.x, tid = threadIdx.x;
+  const int per = (E + nthreads - 1) / nthreads;
+  const int beg = min(E, tid * per), end = min(E, beg + per);
+  int local = 0, lact = 0;
+  for (int e = beg; e < end; ++e) {
+    local += cnt[e];
+    lact += cnt[e] > 0;
+  }
+  int ex, eact, total, tact;
+  block_scan2(local, lact, ex, eact, total, tact, wsum);
+  for (int e = beg; e < end; ++e) {
+    const int c = cnt[e];
+    if (counts) counts[e] = c;
+    if (offsets) offsets[e] = ex;
+    if (cur) cur[e] = ex;
+    if (c > 0) plan[1 + eact++] = e;
+    ex += c;
+  }
+  if (tid == 0) {
+    if (offsets) offsets[E] = total;
+    plan[0] = tact;
+  }
+}
+
+// Stable counting sort of the npairs pairs by expert; block of any size.
+__device__ void bucket_block(const int32_t* idx, int npairs, int E, int32_t* counts,
+                             int32_t* offsets, int32_t* entries, int32_t* plan, int* err,
+                             BucketSmem s) {
+  const int tid = threadIdx.x, nthreads = blockDim.x;
+  const int lane = tid & 31, warp = tid >> 5, nwarps = nthreads >> 5;
+  for (int e = tid; e < E; e += nthreads) s.cnt[e] = 0;
+  for (int i = tid; i < nwarps * E; i += nthreads) s.hist[i] = 0;
+  __syncthreads();
+  for (int p = tid; p < npairs; p += nthreads) {
+    const int e = idx[p];
+    if (e >= 0 && e < E) atomicAdd(&s.cnt[e], 1);
+    else latch_error(err, MOE_ERR_DEVICE_DATA, p);
+  }
+  __syncthreads();
+  offsets_and_plan(s.cnt, E, counts, offsets, plan, s.cur, s.wsum);
+  __syncthreads();
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = 0; base < npairs; base += nthreads) {
+    const int p = base + tid;
+    int e = p < npairs ? idx[p] : -1;
+    const bool valid = e >= 0 && e < E;
+    const unsigned grp = __match_any_sync(kFull, valid ? e : (E + lane));
+    const int rank = __popc(grp & lt_mask);
+    const int gcnt = __popc(grp);
+    if (valid && rank == 0) s.hist[warp * E + e] = uint8_t(gcnt);
+    __syncthreads();
+    if (valid) {
+      int prefix = 0;
+      for (int w = 0; w < warp; ++w) prefix += s.hist[w * E + e];
+      entries[s.cur[e] + prefix + rank] = p;
+    }
+    __syncthreads();
+    if (valid && rank == 0) {
+      atomicAdd(&s.cur[e], gcnt);
+      s.hist[warp * E + e] = 0;
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------- kernels ---
+template <int TT>
+__global__ void __launch_bounds__(kRouteThreads) k_route_logits(RouteArgs a, int fuse_tail) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  pdl_wait();
+  pdl_trigger();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int H = a.H;
+  const int t0 = blockIdx.y * TT;
+  const int nt = min(TT, a.T - t0);
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);           // [TT][H] bf16
+  float* red = reinterpret_cast<float*>(smem + size_t(TT) * H * 2);  // [8][TT]
+  // stage the token rows (16-byte vectors; H % 32 == 0)
+  {
+    const int vec_per_row = H / 8;
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + size_t(t0) * H);
+    uint4* dst = reinterpret_cast<uint4*>(xs);
+    for (int i = tid; i < nt * vec_per_row; i += kRouteThreads) dst[i] = __ldg(src + i);
+  }
+  __syncthreads();
+  const int e = blockIdx.x * 2 + (warp >> 2);
+  const int quarter = warp & 3;
+  const int qlen = H / 4;  // multiple of 8
+  float acc[TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) acc[t] = 0.f;
+  if (e < a.E) {
+    const float* wrow = a.w_router + size_t(e) * H + quarter * qlen;
+    const uint16_t* xq = xs + quarter * qlen;
+    for (int c = lane * 4; c < qlen; c += 128) {
+      const float4 wv = __ldg(reinterpret_cast<const float4*>(wrow + c));
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        if (t < nt) {
+          const uint2 xv = *reinterpret_cast<const uint2*>(xq + size_t(t) * H + c);
+          acc[t] = fmaf(bf16_bits_to_f32(xv.x & 0xffffu), wv.x, acc[t]);
+          acc[t] = fmaf(bf16_bits_to_f32(xv.x >> 16), wv.y, acc[t]);
+          acc[t] = fmaf(bf16_bits_to_f32(xv.y & 0xffffu), wv.z, acc[t]);
+          acc[t] = fmaf(bf16_bits_to_f32(xv.y >> 16), wv.w, acc[t]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < TT; ++t) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) acc[t] += __shfl_xor_sync(kFull, acc[t], off);
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int t = 0; t < TT; ++t) red[warp * TT + t] = acc[t];
+  }
+  __syncthreads();
+  if (tid < 2 * TT) {
+    const int pe = tid / TT, t = tid % TT;
+    const int ee = blockIdx.x * 2 + pe;
+    if (ee < a.E && t < nt) {
+      const float* r = red + (pe * 4) * TT + t;
+      float s = ((r[0] + r[TT]) + r[2 * TT]) + r[3 * TT];
+      if (a.bias) s += __ldg(a.bias + ee);
+      a.logits[size_t(t0 + t) * a.E + ee] = s;
+    }
+  }
+  if (!fuse_tail) return;
+  // ---- the last CTA to arrive routes the whole batch ----
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned total = gridDim.x * gridDim.y;
+    s_last = atomicAdd(a.counter, 1u) == total - 1u;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  int32_t* idx_s = reinterpret_cast<int32_t*>(smem);  // reuse: [T*k]
+  topk_block(a, idx_s);
+  __syncthreads();
+  BucketSmem bs = bucket_smem(smem + align_up16(size_t(a.T) * a.k * 4), a.E, kRouteThreads / 32);
+  bucket_block(idx_s, a.T * a.k, a.E, a.counts, a.offsets, a.entries, a.plan, a.err, bs);
+  if (tid == 0) *a.counter = 0u;
+}
+
+__global__ void __launch_bounds__(kRouteThreads) k_topk(RouteArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5;
+  const int t = blockIdx.x * (kRouteThreads / 32) + warp;
+  if (t >= a.T) return;
+  dispatch_nv(a.E, [&]<int NV>() {
+    topk_warp<NV>(a.logits + size_t(t) * a.E, a.E, a.k, a.idx + size_t(t) * a.k,
+                  a.w + size_t(t) * a.k, nullptr);
+  });
+}
+
+__global__ void __launch_bounds__(kBucketThreads) k_bucket(RouteArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  pdl_wait();
+  pdl_trigger();
+  BucketSmem bs = bucket_smem(smem, a.E, kBucketThreads / 32);
+  bucket_block(a.idx, a.T * a.k, a.E, a.counts, a.offsets, a.entries, a.plan, a.err, bs);
+}
+
+// plan[] from caller-provided offsets (component API path).
+__global__ void __launch_bounds__(kBucketThreads) k_plan(RouteArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  pdl_wait();
+  pdl_trigger();
+  int* cnt = reinterpret_cast<int*>(smem);
+  int* wsum = cnt + a.E;
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+    const int c = __ldg(a.offsets + e + 1) - __ldg(a.offsets + e);
+    if (c < 0) latch_error(a.err, MOE_ERR_DEVICE_DATA, e);
+    cnt[e] = c < 0 ? 0 : c;
+  }
+  __syncthreads();
+  offsets_and_plan(cnt, a.E, nullptr, nullptr, a.plan, nullptr, wsum);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------- launchers ---
+static size_t route_smem(int TT, int H) { return size_t(TT) * H * 2 + 8 * TT * 4; }
+
+cudaError_t launch_route_logits(const RouteArgs& a, bool fuse_tail, cudaStream_t st) {
+  const int TT = a.T <= 1 ? 1 : (a.T <= 2 ? 2 : (a.T <= 4 ? 4 : 8));
+  size_t smem = route_smem(TT, a.H);
+  if (fuse_tail) {
+    const size_t tail = align_up16(size_t(a.T) * a.k * 4) + bucket_smem_bytes(a.E, kRouteThreads);
+    smem = smem > tail ? smem : tail;
+  }
+  dim3 grid((a.E + 1) / 2, (a.T + TT - 1) / TT);
+  cudaError_t err = cudaSuccess;
+  auto go = [&](auto kern) {
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (err == cudaSuccess)
+      err = launch_pdl(kern, grid, dim3(kRouteThreads), smem, st, a, int(fuse_tail));
+  };
+  switch (TT) {
+    case 1: go(k_route_logits<1>); break;
+    case 2: go(k_route_logits<2>); break;
+    case 4: go(k_route_logits<4>); break;
+    default: go(k_route_logits<8>); break;
+  }
+  return err;
+}
+
+size_t route_fused_smem(int T, int H, int E, int k) {
+  const int TT = T <= 1 ? 1 : (T <= 2 ? 2 : (T <= 4 ? 4 : 8));
+  const size_t a = route_smem(TT, H);
+  const size_t b = align_up16(size_t(T) * k * 4) + bucket_smem_bytes(E, kRouteThreads);
+  return a > b ? a : b;
+}
+
+cudaError_t launch_topk(const RouteArgs& a, cudaStream_t st) {
+  const int wpb = kRouteThreads / 32;
+  return launch_pdl(k_topk, dim3((a.T + wpb - 1) / wpb), dim3(kRouteThreads), 0, st, a);
+}
+
+cudaError_t launch_bucket(const RouteArgs& a, cudaStream_t st) {
+  const size_t smem = bucket_smem_bytes(a.E, kBucketThreads);
+  cudaError_t err =
+      cudaFuncSetAttribute(k_bucket, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (err != cudaSuccess) return err;
+  return launch_pdl(k_bucket, dim3(1), dim3(kBucketThreads), smem, st, a);
+}
+
+cudaError_t launch_plan(const RouteArgs& a, cudaStream_t st) {
+  const size_t smem = size_t(a.E) * 4 + 2 * 33 * 4;
+  return launch_pdl(k_plan, dim3(1), dim3(kBucketThreads), smem, st, a);
+}
+
+}  // namespace moe

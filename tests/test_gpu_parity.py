@@ -1,0 +1,275 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI.
+
+Tolerances: integer/index work bit-exact (route indices outside near-ties,
+bucket counts/offsets/entries, MXFP4 codes); combine weights within 1e-5;
+bf16 layer outputs within rel-L2 2e-3 of the oracle rounded to bf16.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from routed_expert_ffn_fp32_b200 import build, moe, synth
+
+from helpers import (TOL_W, TOL_Y, bits_np, check_routing, dev_layer, gpu_layer, rel_l2,
+                     route_depth, to_dev_bits)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    moe.load_library()
+
+
+def cfg_of(name, **kw):
+    return dataclasses.replace(synth.CONFIGS[name], **kw)
+
+
+# ------------------------------------------------------------ MXFP4 codes ---
+def test_decode_exhaustive_codes_and_scales():
+    rows = 16
+    q = np.tile(np.arange(256, dtype=np.uint8), (rows, 1))           # K = 512 per row
+    s = np.arange(256, dtype=np.uint8).reshape(rows, 16)              # every scale byte once
+    out = torch.empty((rows, 512), dtype=torch.float32, device="cuda")
+    moe.moe_decode_mxfp4(torch.from_numpy(q).cuda(), torch.from_numpy(s).cuda(), 512, out)
+    got = out.cpu().numpy()
+    with np.errstate(over="ignore"):
+        want = O.decode_mxfp4(q, s, 512).astype(np.float32)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    np.testing.assert_array_equal(got[ok], want[ok])
+    np.testing.assert_array_equal(np.signbit(got[ok]), np.signbit(want[ok]))
+
+
+def test_act_quant_matches_oracle():
+    rng = np.random.default_rng(3)
+    rows, K = 64, 256
+    v = (rng.normal(size=(rows, K)) * 10.0 ** rng.integers(-6, 4, size=(rows, 1))).astype(np.float32)
+    v[0, :32] = 0.0
+    v[1, :32] = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0] * 4, np.float32)
+    v[2, :32] = -v[1, :32]
+    v[3, :32] = 1e-40                                                 # subnormal block
+    q = torch.empty((rows, K // 2), dtype=torch.uint8, device="cuda")
+    s = torch.empty((rows, K // 32), dtype=torch.uint8, device="cuda")
+    moe.moe_act_quant_mxfp4(torch.from_numpy(v).cuda(), q, s)
+    qg, sg = q.cpu().numpy(), s.cpu().numpy()
+    qo, so = O.quantise_mxfp4_rows(v.astype(np.float64))
+    np.testing.assert_array_equal(sg, so)
+    np.testing.assert_array_equal(O.decode_mxfp4(qg, sg, K), O.decode_mxfp4(qo, so, K))
+
+
+# ---------------------------------------------------------------- routing ---
+ROUTE_CASES = [("tiny_h256_i128_e8_k2", 4), ("decode_h4096_i1408_e64_k2", 1),
+               ("decode_h4096_i1408_e64_k2", 5), ("finegrained_h4096_i2048_e256_k8_shared", 1),
+               ("finegrained_h4096_i2048_e256_k8_shared", 5),
+               ("finegrained_h4096_i2048_e256_k8_shared", 37),
+               ("prefill_h4096_i2048_e256_k8_shared_zipf1.2", 300)]
+
+
+@pytest.mark.parametrize("name,T", ROUTE_CASES)
+def test_route_topk(name, T):
+    cfg = synth.CONFIGS[name]
+    x = synth.activations(cfg, 0, T)
+    W_r, bias = synth.router(cfg, 0)
+    shape = moe.shape_of(T, cfg.H, cfg.I, cfg.E, cfg.k)
+    ws = moe.make_workspace(shape, moe.MOE_PATH_GEMV)
+    idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
+    logits = torch.empty((T, cfg.E), dtype=torch.float32, device="cuda")
+    moe.moe_route_topk(to_dev_bits(x), torch.from_numpy(W_r).cuda(),
+                       None if bias is None else torch.from_numpy(bias).cuda(), shape, idx, w, ws,
+                       logits_out=logits)
+    xf = O.bf16_bits_to_f64(x)
+    lref = O.router_logits(xf, W_r, bias)
+    iref, wref = O.route_topk(lref, cfg.k)
+    # logits within the float32 error bound of the kernel's summation
+    u = 2.0 ** -24
+    d = route_depth(cfg.H)
+    bound = d * u / (1 - d * u) * (np.abs(xf) @ np.abs(W_r.astype(np.float64)).T) + 2 * u * np.abs(lref)
+    if bias is not None:
+        bound += u * np.abs(bias)
+    assert (np.abs(logits.cpu().numpy() - lref) <= bound).all()
+    ref = {"logits": lref, "idx": iref, "w": wref}
+    L = {"x": x, "W_r": W_r, "bias": bias}
+    check_routing(L, ref, idx.cpu().numpy(), w.cpu().numpy(), cfg.k, cfg.H)
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 8, 2), (5, 64, 2), (37, 256, 8), (4096, 256, 8),
+                                   (4096, 1024, 16), (3, 1, 1), (1000, 7, 7)])
+def test_bucket_bit_exact(T, E, k):
+    rng = np.random.default_rng(T * 7 + E)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    shape = moe.shape_of(T, 64, 64, E, k)
+    ws = moe.make_workspace(shape, moe.MOE_PATH_GEMV)
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    entries = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    moe.moe_bucket(torch.from_numpy(idx).cuda(), shape, counts, offsets, entries, ws)
+    c, o, e = O.bucket_by_expert(idx, E)
+    np.testing.assert_array_equal(counts.cpu().numpy(), c)
+    np.testing.assert_array_equal(offsets.cpu().numpy(), o)
+    np.testing.assert_array_equal(entries.cpu().numpy(), e)
+    assert moe.moe_get_error(ws) == 0
+
+
+def test_bucket_bad_index_latches_error():
+    T, E, k = 6, 8, 2
+    idx = np.array([[0, 1], [2, 9], [3, 4], [5, -1], [6, 7], [1, 0]], np.int32)
+    shape = moe.shape_of(T, 64, 64, E, k)
+    ws = moe.make_workspace(shape, moe.MOE_PATH_GEMV)
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    entries = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
+    moe.moe_bucket(torch.from_numpy(idx).cuda(), shape, counts, offsets, entries, ws)
+    assert moe.moe_get_error(ws) == moe.MOE_ERR_DEVICE_DATA
+    assert moe.moe_get_error(ws) == 0                       # cleared by the read
+    valid = idx.copy()
+    keep = (valid >= 0) & (valid < E)
+    assert counts.cpu().numpy().sum() == keep.sum()
+    assert offsets.cpu().numpy()[-1] == keep.sum()
+
+
+# ------------------------------------------------------------ expert FFN ----
+@pytest.mark.parametrize("name,T", [("tiny_h256_i128_e8_k2", 4), ("decode_h4096_i1408_e64_k2", 5),
+                                    ("finegrained_h4096_i2048_e256_k8_shared", 5)])
+@pytest.mark.parametrize("precision", [moe.MOE_ACT_EXACT, moe.MOE_ACT_MXFP4])
+def test_expert_ffn_partials(name, T, precision):
+    cfg = synth.CONFIGS[name]
+    L = synth.layer(cfg, 0, T)
+    mode = "mxfp4_act" if precision == moe.MOE_ACT_MXFP4 else "exact"
+    ref = O.layer_forward(L["x"], L["W_r"], L["bias"], L["experts"], L["shared"], cfg.k, mode)
+    D = dev_layer(L)
+    shape = moe.shape_of(T, cfg.H, cfg.I, cfg.E, cfg.k)
+    has_sh = D["shared"] is not None
+    ws = moe.make_workspace(shape, moe.MOE_PATH_GEMV, precision, has_sh)
+    rows = T * cfg.k + (T if has_sh else 0)
+    partial = torch.zeros((rows, cfg.H), dtype=torch.float32, device="cuda")
+    moe.moe_expert_ffn_mxfp4(D["experts"], D["shared"], D["x"],
+                             torch.from_numpy(ref["offsets"]).cuda(),
+                             torch.from_numpy(ref["entries"]).cuda(), shape, partial, ws,
+                             moe.MOE_PATH_GEMV, precision)
+    got = partial.cpu().numpy()
+    assert moe.moe_get_error(ws) == 0
+    tol = 1e-4 if precision == moe.MOE_ACT_EXACT else 2e-3
+    for r in range(rows):
+        assert rel_l2(got[r], ref["partial"][r]) < tol, r
+
+
+def test_combine_matches_fp64():
+    rng = np.random.default_rng(11)
+    T, H, k = 7, 512, 3
+    partial = rng.normal(size=(T * k + T, H)).astype(np.float32)
+    w = rng.random(size=(T, k)).astype(np.float32)
+    w /= w.sum(1, keepdims=True)
+    shape = moe.shape_of(T, H, 64, 8, k)
+    for has_sh in (0, 1):
+        y = torch.empty((T, H), dtype=torch.int16, device="cuda")
+        moe.moe_combine(torch.from_numpy(partial).cuda(), torch.from_numpy(w).cuda(), shape, has_sh, y)
+        ref = np.zeros((T, H))
+        for t in range(T):
+            for j in range(k):
+                ref[t] += np.float64(w[t, j]) * partial[t * k + j]
+            if has_sh:
+                ref[t] += partial[T * k + t]
+        got = O.bf16_bits_to_f64(bits_np(y))
+        want = O.bf16_bits_to_f64(O.f64_to_bf16_bits(ref))
+        # at most one bf16 ulp apart (float32 vs exact sums may round differently)
+        assert (np.abs(got - want) <= np.abs(want) * 2.0 ** -7 + 1e-30).all()
+        assert rel_l2(got, want) < TOL_Y
+
+
+# ------------------------------------------------------------- the layer ----
+LAYER_CASES = [
+    ("tiny_h256_i128_e8_k2", 4), ("tiny_h256_i128_e8_k2", 1), ("tiny_h256_i128_e8_k2", 33),
+    ("decode_h4096_i1408_e64_k2", 1), ("decode_h4096_i1408_e64_k2", 5),
+    ("finegrained_h4096_i2048_e256_k8_shared", 1), ("finegrained_h4096_i2048_e256_k8_shared", 5),
+]
+
+
+@pytest.mark.parametrize("name,T", LAYER_CASES)
+def test_layer_forward(name, T):
+    cfg = synth.CONFIGS[name]
+    L = synth.layer(cfg, 0, T)
+    ref = O.layer_forward(L["x"], L["W_r"], L["bias"], L["experts"], L["shared"], cfg.k)
+    out = gpu_layer(L, dev_layer(L), cfg)
+    check_routing(L, ref, out["idx"], out["w"], cfg.k, cfg.H)
+    want = O.bf16_bits_to_f64(ref["y_bf16"])
+    got = O.bf16_bits_to_f64(out["y"])
+    assert rel_l2(got, want) < TOL_Y
+    assert rel_l2(got, ref["y"]) < TOL_Y
+
+
+def test_layer_forward_mxfp4_act_mode():
+    cfg = synth.TINY
+    L = synth.layer(cfg, 2, 16)
+    ref = O.layer_forward(L["x"], L["W_r"], L["bias"], L["experts"], L["shared"], cfg.k, "mxfp4_act")
+    out = gpu_layer(L, dev_layer(L), cfg, moe.MOE_PATH_GEMV, moe.MOE_ACT_MXFP4)
+    assert rel_l2(O.bf16_bits_to_f64(out["y"]), O.bf16_bits_to_f64(ref["y_bf16"])) < TOL_Y
+
+
+EDGE = [
+    # (H, I, E, k, T, shared, bias)
+    (96, 32, 4, 4, 3, False, True),       # k == E, odd block counts
+    (64, 64, 1, 1, 2, True, False),       # a single expert
+    (8192, 256, 16, 2, 3, False, False),  # wide rows (two blocks per lane)
+    (512, 4096, 8, 3, 5, True, True),     # wide down rows
+    (256, 128, 1024, 16, 9, False, True), # many experts, k = 16
+    (128, 96, 32, 1, 40, False, True),    # k = 1, unfused routing (T > 32)
+]
+
+
+@pytest.mark.parametrize("H,I,E,k,T,shared,bias", EDGE)
+def test_layer_edge_shapes(H, I, E, k, T, shared, bias):
+    cfg = synth.LayerConfig("edge", H, I, E, k, T, 0.05, 1.0 if bias else None, shared)
+    L = synth.layer(cfg, 5, T)
+    ref = O.layer_forward(L["x"], L["W_r"], L["bias"], L["experts"], L["shared"], k)
+    out = gpu_layer(L, dev_layer(L), cfg)
+    check_routing(L, ref, out["idx"], out["w"], k, H)
+    assert rel_l2(O.bf16_bits_to_f64(out["y"]), O.bf16_bits_to_f64(ref["y_bf16"])) < TOL_Y
+
+
+def test_one_hot_and_zero_experts():
+    cfg = synth.LayerConfig("onehot", 256, 128, 8, 1, 6, 0.05, None, True)
+    L = synth.layer(cfg, 9)
+    L["W_r"] = np.zeros_like(L["W_r"])
+    L["bias"] = np.zeros(8, np.float32)
+    L["bias"][5] = 50.0
+    ref = O.layer_forward(L["x"], L["W_r"], L["bias"], L["experts"], L["shared"], 1)
+    out = gpu_layer(L, dev_layer(L), cfg)
+    assert (out["idx"][:, 0] == 5).all() and (out["w"] == 1.0).all()
+    assert rel_l2(O.bf16_bits_to_f64(out["y"]), O.bf16_bits_to_f64(ref["y_bf16"])) < TOL_Y
+    L["experts"] = {n: np.zeros_like(a) for n, a in L["experts"].items()}
+    ref = O.layer_forward(L["x"], L["W_r"], L["bias"], L["experts"], L["shared"], 1)
+    out = gpu_layer(L, dev_layer(L), cfg)
+    assert rel_l2(O.bf16_bits_to_f64(out["y"]), O.bf16_bits_to_f64(ref["y_bf16"])) < TOL_Y
+
+
+def test_graph_replay_matches_eager():
+    cfg = synth.DECODE64
+    L = synth.layer(cfg, 0, 5)
+    D = dev_layer(L)
+    shape = moe.shape_of(5, cfg.H, cfg.I, cfg.E, cfg.k)
+    ws = moe.make_workspace(shape, moe.MOE_PATH_GEMV)
+    y = torch.empty((5, cfg.H), dtype=torch.int16, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        moe.moe_layer_forward(D["x"], D["W_r"], None, D["experts"], None, shape, y, ws)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            moe.moe_layer_forward(D["x"], D["W_r"], None, D["experts"], None, shape, y, ws)
+    eager = bits_np(y).copy()
+    x2 = synth.activations(cfg, 1, 5)
+    D["x"].copy_(to_dev_bits(x2))
+    g.replay()
+    torch.cuda.synchronize()
+    ref = O.layer_forward(x2, L["W_r"], None, L["experts"], None, cfg.k)
+    assert rel_l2(O.bf16_bits_to_f64(bits_np(y)), O.bf16_bits_to_f64(ref["y_bf16"])) < TOL_Y
+    D["x"].copy_(to_dev_bits(L["x"]))
+    g.replay()
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(bits_np(y), eager)       # deterministic
