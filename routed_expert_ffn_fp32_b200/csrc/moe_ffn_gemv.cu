@@ -32,7 +32,6 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
-constexpr int kPiece = 64;  // units per epilogue piece
 
 // Arithmetic policies for one 32-element block dot product.
 enum Policy : int {
@@ -121,11 +120,6 @@ __device__ __forceinline__ void load_block_f32(const float* row, int b, float (&
     f[4 * q + 3] = v.w;
   }
 }
-
-template <int POL>
-struct BlockW {
-  uint32_t h[16];  // f16x2 weight pairs
-};
 
 __device__ __forceinline__ void decode_codes(const uint4& c, uint32_t (&h)[16]) {
   uint32_t t[4];
@@ -222,32 +216,115 @@ __device__ __forceinline__ int token_of(const FfnArgs& a, const VExpert& ve, int
   return ve.rows ? ve.rows[r] / a.k : r;
 }
 
+// ---------------------------------------------------------------------------
+// Asynchronous global -> shared copies (cp.async): each lane streams its own
+// 16-byte code chunks into a per-warp ring of stages, so several stages of
+// weights are in flight while the warp computes on an earlier one.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void group_barrier(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+constexpr int kStages = 4;        // ring depth per warp
+constexpr int kSlots = 8;         // 512-byte code chunks per stage per warp
+constexpr int kChunk = 512;       // one warp-wide 16-byte-per-lane row slice
+constexpr int kStageBytes = kSlots * (kChunk + 32);
+constexpr int kRingBytes = kStages * kStageBytes;
+constexpr int kPartBytes = 2 * kWarps * 32 * 4;
+constexpr int kGemvSmem = kWarps * kRingBytes + kPartBytes;
+
+template <int PHASE>
+struct PhaseCfg {
+  static constexpr int NPROJ = PHASE == 0 ? 2 : 1;
+  // gate/up: token rows enter as f16 (exact for bf16 inputs); down: the
+  // float32 SwiGLU output enters as it is.
+  static constexpr int POL = PHASE == 0 ? kMixed : kF32x2;
+};
+
+struct Worker {
+  int KS, NG, grp, gl, lstride, nb, bar_id, bar_n;
+  int warp, lane;
+  unsigned char* ring;  // this warp's stages
+  float* part;          // [2][kWarps][32]
+  int fast_scales;      // scale rows 4-byte aligned: stage them with cp.async
+  unsigned parity;      // stage counter (selects the part buffer)
+};
+
 // One virtual expert, units [r0, r1), tokens [t0, t0 + nt) of its bucket.
-template <int PHASE, int POL, int RC, int BPL>
-__device__ void run_span(const FfnArgs& a, const VExpert& ve, int r0, int r1, int t0, int nt,
-                         int KS, float* part) {
-  constexpr int NPROJ = PHASE == 0 ? 2 : 1;
-  // units per group: at most 16 code loads in flight per lane, at most 32
-  // accumulators (the butterfly reduction works on a power of two <= 32)
-  constexpr int UG_LOAD = 16 / (NPROJ * BPL) > 0 ? 16 / (NPROJ * BPL) : 1;
+template <int PHASE, int BPL, int RC>
+__device__ void run_segment(const FfnArgs& a, const VExpert& ve, int r0, int r1, int t0, int nt,
+                            Worker& wk) {
+  using C = PhaseCfg<PHASE>;
+  constexpr int NPROJ = C::NPROJ;
+  constexpr int POL = C::POL;
+  constexpr int UG_SM = kSlots / (NPROJ * BPL) > 0 ? kSlots / (NPROJ * BPL) : 1;
   constexpr int UG_ACC = 32 / (NPROJ * RC) > 0 ? 32 / (NPROJ * RC) : 1;
-  constexpr int UG = UG_LOAD < UG_ACC ? UG_LOAD : UG_ACC;
+  constexpr int UG = UG_SM < UG_ACC ? UG_SM : UG_ACC;
   constexpr int NVAL = UG * NPROJ * RC;
   static_assert((NVAL & (NVAL - 1)) == 0 && NVAL <= 32, "NVAL must be a power of two <= 32");
   const int K = PHASE == 0 ? a.H : a.I;
-  const int ROWS = PHASE == 0 ? a.I : a.H;
-  const int nb = K / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int NG = kWarps / KS;
-  const int grp = warp / KS;
-  const int gl = (warp % KS) * 32 + lane;  // lane index within the K group
-  const int lstride = 32 * KS;
+  const size_t rowq = size_t(K) / 2;
+  const int nb = wk.nb, lane = wk.lane;
+  const int nunits = r1 - r0;
+  const int nst = (nunits + UG - 1) / UG;
+  const int span0 = (wk.warp % wk.KS) * 32;  // first block of this warp's K slice
 
-  // token rows -> registers
+  auto issue = [&](int st) {
+    if (st < nst) {
+      unsigned char* stage = wk.ring + (st % kStages) * kStageBytes;
+#pragma unroll
+      for (int u = 0; u < UG; ++u) {
+        const int row = r0 + st * UG + u;
+        if (row < r1) {
+#pragma unroll
+          for (int pj = 0; pj < NPROJ; ++pj) {
+#pragma unroll
+            for (int m = 0; m < BPL; ++m) {
+              const int slot = (u * NPROJ + pj) * BPL + m;
+              const int b = wk.gl + m * wk.lstride;
+              if (b < nb)
+                cp_async16(stage + slot * kChunk + lane * 16,
+                           ve.q[pj] + size_t(row) * rowq + size_t(b) * 16);
+              if (wk.fast_scales) {
+                const int sb = span0 + m * wk.lstride;  // first block of the 32-byte span
+                if (lane < 8 && sb + 4 * lane + 4 <= nb)
+                  cp_async4(stage + kSlots * kChunk + slot * 32 + lane * 4,
+                            ve.s[pj] + size_t(row) * nb + sb + 4 * lane);
+              }
+            }
+          }
+        }
+      }
+    }
+    cp_async_commit();
+  };
+
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) issue(s);
+
+  // token rows -> registers (overlaps the first stages in flight)
   XReg<POL> xr[BPL][RC];
 #pragma unroll
   for (int m = 0; m < BPL; ++m) {
-    const int b = gl + m * lstride;
+    const int b = wk.gl + m * wk.lstride;
 #pragma unroll
     for (int t = 0; t < RC; ++t) {
       float f[32];
@@ -266,97 +343,102 @@ __device__ void run_span(const FfnArgs& a, const VExpert& ve, int r0, int r1, in
     }
   }
 
-  const size_t rowq = size_t(K) / 2;
-  for (int p0 = r0; p0 < r1; p0 += kPiece) {
-    const int np = min(kPiece, r1 - p0);
-    const int gbeg = (grp * np) / NG, gend = ((grp + 1) * np) / NG;
-    for (int g = gbeg; g < gend; g += UG) {
-      float acc[NVAL];
+  for (int st = 0; st < nst; ++st) {
+    issue(st + kStages - 1);
+    cp_async_wait<kStages - 1>();
+    __syncwarp();
+    const unsigned char* stage = wk.ring + (st % kStages) * kStageBytes;
+    float acc[NVAL];
 #pragma unroll
-      for (int i = 0; i < NVAL; ++i) acc[i] = 0.f;
-      uint4 cq[UG][NPROJ][BPL];
-      uint32_t cs[UG][NPROJ][BPL];
+    for (int i = 0; i < NVAL; ++i) acc[i] = 0.f;
 #pragma unroll
-      for (int u = 0; u < UG; ++u) {
-        const int row = p0 + g + u;
-        const bool uv = (g + u) < gend;
+    for (int u = 0; u < UG; ++u) {
+      if (r0 + st * UG + u < r1) {
 #pragma unroll
         for (int pj = 0; pj < NPROJ; ++pj) {
 #pragma unroll
           for (int m = 0; m < BPL; ++m) {
-            const int b = gl + m * lstride;
-            if (uv && b < nb) {
-              cq[u][pj][m] = ldg_stream(ve.q[pj] + size_t(row) * rowq + size_t(b) * 16);
-              cs[u][pj][m] = ldg_u8(ve.s[pj] + size_t(row) * nb + b);
-            } else {
-              cq[u][pj][m] = make_uint4(0, 0, 0, 0);
-              cs[u][pj][m] = 127u;
+            const int slot = (u * NPROJ + pj) * BPL + m;
+            const int b = wk.gl + m * wk.lstride;
+            if (b < nb) {
+              const uint4 c = *reinterpret_cast<const uint4*>(stage + slot * kChunk + lane * 16);
+              const int row = r0 + st * UG + u;
+              const uint32_t sbyte =
+                  wk.fast_scales ? uint32_t(stage[kSlots * kChunk + slot * 32 + lane])
+                                 : ldg_u8(ve.s[pj] + size_t(row) * nb + b);
+              uint32_t w[16];
+              decode_codes(c, w);
+              const float sc = e8m0_to_f32(sbyte);
+#pragma unroll
+              for (int t = 0; t < RC; ++t) {
+                const float bs = block_dot<POL>(w, xr[m][t]);
+                float& dst = acc[(u * NPROJ + pj) * RC + t];
+                dst = fmaf(sc, bs, dst);
+              }
             }
           }
         }
       }
-#pragma unroll
-      for (int u = 0; u < UG; ++u) {
-#pragma unroll
-        for (int pj = 0; pj < NPROJ; ++pj) {
-#pragma unroll
-          for (int m = 0; m < BPL; ++m) {
-            uint32_t w[16];
-            decode_codes(cq[u][pj][m], w);
-            const float sc = e8m0_to_f32(cs[u][pj][m]);
-#pragma unroll
-            for (int t = 0; t < RC; ++t) {
-              const float bs = block_dot<POL>(w, xr[m][t]);
-              float& dst = acc[(u * NPROJ + pj) * RC + t];
-              dst = fmaf(sc, bs, dst);
-            }
-          }
+    }
+    const float tot = transpose_reduce<NVAL>(acc, lane);
+    float* part = wk.part + (wk.parity & 1u) * (kWarps * 32);
+    if (lane < NVAL) part[wk.warp * 32 + lane] = tot;
+    group_barrier(wk.bar_id, wk.bar_n);
+    // finalize: the KS warps of the group add their K-slice sums
+    const int q = (wk.warp % wk.KS) * 32 + lane;
+    if (q < UG * RC) {
+      const int u = q / RC, t = q % RC;
+      const int row = r0 + st * UG + u;
+      if (row < r1 && t < nt) {
+        float s0 = 0.f, s1 = 0.f;
+        for (int w = 0; w < wk.KS; ++w) {
+          const float* pw = part + (wk.grp * wk.KS + w) * 32;
+          s0 += pw[(u * NPROJ + 0) * RC + t];
+          if constexpr (NPROJ == 2) s1 += pw[(u * NPROJ + 1) * RC + t];
+        }
+        const int orow = out_row(a, ve, t0 + t);
+        if constexpr (PHASE == 0) {
+          a.h[size_t(orow) * a.I + row] = s0 / (1.f + expf(-s0)) * s1;  // silu(g) * u
+        } else {
+          a.partial[size_t(orow) * a.H + row] = s0;
         }
       }
-      const float tot = transpose_reduce<NVAL>(acc, lane);
-      if (lane < NVAL) {
-        const int t = lane % RC;
-        const int pj = (lane / RC) % NPROJ;
-        const int u = lane / (RC * NPROJ);
-        if (g + u < gend) part[((warp * kPiece + g + u) * NPROJ + pj) * RC + t] = tot;
-      }
     }
-    __syncthreads();
-    // epilogue: add the KS warps' partial sums of each unit
-    for (int q = threadIdx.x; q < np * nt; q += kThreads) {
-      const int uix = q % np, t = q / np;
-      int owner = 0;
-      for (int gi = 1; gi < NG; ++gi)
-        if ((gi * np) / NG <= uix) owner = gi;
-      float s0 = 0.f, s1 = 0.f;
-      for (int w = owner * KS; w < owner * KS + KS; ++w) {
-        s0 += part[((w * kPiece + uix) * NPROJ + 0) * RC + t];
-        if constexpr (NPROJ == 2) s1 += part[((w * kPiece + uix) * NPROJ + 1) * RC + t];
-      }
-      const int orow = out_row(a, ve, t0 + t);
-      if constexpr (PHASE == 0) {
-        const float hval = s0 / (1.f + expf(-s0)) * s1;  // silu(g) * u
-        a.h[size_t(orow) * a.I + p0 + uix] = hval;
-      } else {
-        a.partial[size_t(orow) * a.H + p0 + uix] = s0;
-      }
-    }
-    __syncthreads();
+    ++wk.parity;
   }
-  (void)ROWS;
+  cp_async_wait<0>();
+  __syncwarp();
 }
 
-template <int PHASE, int POL, int RCMAX, int BPL>
-__global__ void __launch_bounds__(kThreads) k_ffn_gemv(FfnArgs a, int KS) {
-  __shared__ float part[kWarps * kPiece * (PHASE == 0 ? 2 : 1) * RCMAX];
+template <int PHASE, int BPL, int RCMAX>
+__global__ void __launch_bounds__(kThreads) k_ffn_gemv(FfnArgs a, int KS, int fast_scales) {
+  extern __shared__ __align__(128) unsigned char smem[];
   pdl_wait();
   pdl_trigger();
+  Worker wk;
+  wk.lane = threadIdx.x & 31;
+  wk.warp = threadIdx.x >> 5;
+  wk.KS = KS;
+  wk.NG = kWarps / KS;
+  wk.grp = wk.warp / KS;
+  wk.gl = (wk.warp % KS) * 32 + wk.lane;
+  wk.lstride = 32 * KS;
+  wk.nb = (PHASE == 0 ? a.H : a.I) / 32;
+  wk.bar_id = 1 + wk.grp;
+  wk.bar_n = 32 * KS;
+  wk.ring = smem + wk.warp * kRingBytes;
+  wk.part = reinterpret_cast<float*>(smem + kWarps * kRingBytes);
+  wk.fast_scales = fast_scales;
+  wk.parity = 0;
+
   const int nA = a.plan[0];
   const int nV = nA + (a.has_shared ? 1 : 0);
   const int ROWS = PHASE == 0 ? a.I : a.H;
   const long long U = (long long)nV * ROWS;
-  const long long ub = U * blockIdx.x / gridDim.x;
-  const long long ue = U * (blockIdx.x + 1) / gridDim.x;
+  const long long nW = (long long)gridDim.x * wk.NG;
+  const long long worker = (long long)blockIdx.x * wk.NG + wk.grp;
+  const long long ub = U * worker / nW;
+  const long long ue = U * (worker + 1) / nW;
   long long u = ub;
   while (u < ue) {
     const int v = int(u / ROWS);
@@ -365,42 +447,69 @@ __global__ void __launch_bounds__(kThreads) k_ffn_gemv(FfnArgs a, int KS) {
     const VExpert ve = vexpert(a, PHASE, v, nA);
     for (int t0 = 0; t0 < ve.R; t0 += RCMAX) {
       const int nt = min(RCMAX, ve.R - t0);
-      // smallest register tile holding the chunk
-      if (RCMAX >= 4 && nt > 2) {
-        run_span<PHASE, POL, (RCMAX >= 4 ? 4 : RCMAX), BPL>(a, ve, r0, r1, t0, nt, KS, part);
+      if (RCMAX >= 8 && nt > 4) {
+        run_segment<PHASE, BPL, (RCMAX >= 8 ? 8 : RCMAX)>(a, ve, r0, r1, t0, nt, wk);
+      } else if (RCMAX >= 4 && nt > 2) {
+        run_segment<PHASE, BPL, (RCMAX >= 4 ? 4 : RCMAX)>(a, ve, r0, r1, t0, nt, wk);
       } else if (RCMAX >= 2 && nt == 2) {
-        run_span<PHASE, POL, (RCMAX >= 2 ? 2 : RCMAX), BPL>(a, ve, r0, r1, t0, nt, KS, part);
+        run_segment<PHASE, BPL, (RCMAX >= 2 ? 2 : RCMAX)>(a, ve, r0, r1, t0, nt, wk);
       } else {
-        run_span<PHASE, POL, 1, BPL>(a, ve, r0, r1, t0, nt, KS, part);
+        run_segment<PHASE, BPL, 1>(a, ve, r0, r1, t0, nt, wk);
       }
     }
     u += r1 - r0;
   }
 }
 
-template <int PHASE, int POL>
-cudaError_t launch_phase(const FfnArgs& a, int grid, cudaStream_t st) {
-  const int K = PHASE == 0 ? a.H : a.I;
+// K split and blocks per lane for a projection of K columns.
+inline void split_of(int K, int& KS, int& BPL) {
   const int nb = K / 32;
-  int KS, BPL;
   if (nb <= 32) { KS = 1; BPL = 1; }
   else if (nb <= 64) { KS = 2; BPL = 1; }
   else if (nb <= 128) { KS = 4; BPL = 1; }
   else if (nb <= 256) { KS = 4; BPL = 2; }
   else { KS = 4; BPL = 4; }
-  // register tile of tokens: at most 4 per pass, fewer for wide rows
-  const int rcmax_cap = BPL == 1 ? 4 : (BPL == 2 ? 2 : 1);
-  int RCMAX = a.T >= 4 ? 4 : (a.T >= 2 ? 2 : 1);
-  if (RCMAX > rcmax_cap) RCMAX = rcmax_cap;
-  const dim3 g(grid), b(kThreads);
-#define MOE_GEMV_CASE(RCM, B)                                                          \
-  if (RCMAX == RCM && BPL == B) return launch_pdl(k_ffn_gemv<PHASE, POL, RCM, B>, g, b, 0, st, a, KS);
+}
+
+// Largest token tile per pass: x registers hold BPL * RC blocks per lane.
+inline int rcmax_of(int PHASE, int T, int BPL) {
+  int cap = PHASE == 0 ? 8 : 4;
+  cap = cap / BPL > 0 ? cap / BPL : 1;
+  const int want = T >= 8 ? 8 : T;
+  int r = 1;
+  while (r < want) r <<= 1;
+  return r < cap ? r : cap;
+}
+
+template <int PHASE, int BPL, int RCMAX>
+cudaError_t launch_one(const FfnArgs& a, int grid, int KS, int fast, cudaStream_t st) {
+  auto kern = k_ffn_gemv<PHASE, BPL, RCMAX>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kGemvSmem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), size_t(kGemvSmem), st, a, KS, fast);
+}
+
+template <int PHASE>
+cudaError_t launch_phase(const FfnArgs& a, int grid, cudaStream_t st) {
+  const int K = PHASE == 0 ? a.H : a.I;
+  int KS, BPL;
+  split_of(K, KS, BPL);
+  const int RCMAX = rcmax_of(PHASE, a.T, BPL);
+  const int fast = (K / 32) % 4 == 0;
+#define MOE_GEMV_CASE(B, R) \
+  if (BPL == B && RCMAX == R) return launch_one<PHASE, B, R>(a, grid, KS, fast, st);
   MOE_GEMV_CASE(1, 1)
-  MOE_GEMV_CASE(2, 1)
-  MOE_GEMV_CASE(4, 1)
   MOE_GEMV_CASE(1, 2)
-  MOE_GEMV_CASE(2, 2)
   MOE_GEMV_CASE(1, 4)
+  MOE_GEMV_CASE(2, 1)
+  MOE_GEMV_CASE(2, 2)
+  MOE_GEMV_CASE(4, 1)
+  if constexpr (PHASE == 0) {
+    MOE_GEMV_CASE(1, 8)
+    MOE_GEMV_CASE(2, 4)
+    MOE_GEMV_CASE(4, 2)
+  }
 #undef MOE_GEMV_CASE
   return cudaErrorInvalidValue;
 }
@@ -439,30 +548,23 @@ __global__ void __launch_bounds__(256) k_combine(const float* partial, const flo
 
 }  // namespace
 
-#ifndef MOE_GEMV_POLICY
-#define MOE_GEMV_POLICY 0
-#endif
-
-int gemv_grid(int phase) {
-  static int occ[2] = {0, 0};
-  const DeviceInfo di = device_info();
-  if (occ[phase] == 0) {
+int gemv_grid() {
+  static int occ = 0;
+  if (occ == 0) {
     int o = 0;
-    if (phase == 0)
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_ffn_gemv<0, MOE_GEMV_POLICY, 4, 1>,
-                                                    kThreads, 0);
-    else
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_ffn_gemv<1, MOE_GEMV_POLICY, 4, 1>,
-                                                    kThreads, 0);
-    occ[phase] = o > 0 ? o : 1;
+    cudaFuncSetAttribute(k_ffn_gemv<0, 1, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kGemvSmem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_ffn_gemv<0, 1, 8>, kThreads, kGemvSmem);
+    occ = o > 0 ? o : 1;
   }
-  return di.sm_count * occ[phase];
+  return device_info().sm_count * occ;
 }
 
 cudaError_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t st) {
-  cudaError_t e = launch_phase<0, MOE_GEMV_POLICY>(a, gemv_grid(0), st);
+  const int grid = gemv_grid();
+  cudaError_t e = launch_phase<0>(a, grid, st);
   if (e != cudaSuccess) return e;
-  return launch_phase<1, MOE_GEMV_POLICY>(a, gemv_grid(1), st);
+  return launch_phase<1>(a, grid, st);
 }
 
 cudaError_t launch_combine(const float* partial, const float* w, int T, int H, int k,

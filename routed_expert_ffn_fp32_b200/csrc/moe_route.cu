@@ -281,16 +281,29 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_logits(RouteArgs a, int
   if (e < a.E) {
     const float* wrow = a.w_router + size_t(e) * H + quarter * qlen;
     const uint16_t* xq = xs + quarter * qlen;
-    for (int c = lane * 4; c < qlen; c += 128) {
-      const float4 wv = __ldg(reinterpret_cast<const float4*>(wrow + c));
+    // eight float4 loads in flight per lane before the arithmetic on them
+    for (int base = lane * 4; base < qlen; base += 128 * 8) {
+      float4 wv[8];
 #pragma unroll
-      for (int t = 0; t < TT; ++t) {
-        if (t < nt) {
-          const uint2 xv = *reinterpret_cast<const uint2*>(xq + size_t(t) * H + c);
-          acc[t] = fmaf(bf16_bits_to_f32(xv.x & 0xffffu), wv.x, acc[t]);
-          acc[t] = fmaf(bf16_bits_to_f32(xv.x >> 16), wv.y, acc[t]);
-          acc[t] = fmaf(bf16_bits_to_f32(xv.y & 0xffffu), wv.z, acc[t]);
-          acc[t] = fmaf(bf16_bits_to_f32(xv.y >> 16), wv.w, acc[t]);
+      for (int j = 0; j < 8; ++j) {
+        const int c = base + 128 * j;
+        wv[j] = c < qlen ? __ldg(reinterpret_cast<const float4*>(wrow + c))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int c = base + 128 * j;
+        if (c < qlen) {
+#pragma unroll
+          for (int t = 0; t < TT; ++t) {
+            if (t < nt) {
+              const uint2 xv = *reinterpret_cast<const uint2*>(xq + size_t(t) * H + c);
+              acc[t] = fmaf(bf16_bits_to_f32(xv.x & 0xffffu), wv[j].x, acc[t]);
+              acc[t] = fmaf(bf16_bits_to_f32(xv.x >> 16), wv[j].y, acc[t]);
+              acc[t] = fmaf(bf16_bits_to_f32(xv.y & 0xffffu), wv[j].z, acc[t]);
+              acc[t] = fmaf(bf16_bits_to_f32(xv.y >> 16), wv[j].w, acc[t]);
+            }
+          }
         }
       }
     }
