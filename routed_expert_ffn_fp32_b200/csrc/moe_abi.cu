@@ -82,13 +82,21 @@ bool valid_path(int32_t path) {
 }
 bool valid_precision(int32_t p) { return p == MOE_ACT_EXACT || p == MOE_ACT_MXFP4; }
 
+// Batches from which AUTO takes the tensor-core path (MXFP4 activations only):
+// below it the weight stream dominates and the CUDA-core GEMV is as fast.
+constexpr int kGemmMinPairs = 512;
+
 // Resolves AUTO; returns MOE_PATH_GEMV or MOE_PATH_GEMM, or -1 if unsupported.
 int resolve_path(int32_t path, int32_t precision, const moe_shape_t& s) {
-  (void)precision;
-  (void)s;
-  if (path == MOE_PATH_GEMM) return -1;  // tensor-core path not available in this build
+  if (path == MOE_PATH_GEMM)
+    return (precision == MOE_ACT_MXFP4 && gemm_supported(s)) ? MOE_PATH_GEMM : -1;
+  if (path == MOE_PATH_AUTO && precision == MOE_ACT_MXFP4 && s.T * s.k >= kGemmMinPairs &&
+      gemm_supported(s))
+    return MOE_PATH_GEMM;
   return MOE_PATH_GEMV;
 }
+
+GemmBuffers gemm_buffers(void* ws, const WsLayout& L, int E);
 
 template <typename T>
 T* at(void* ws, size_t off) {
@@ -96,6 +104,17 @@ T* at(void* ws, size_t off) {
 }
 
 constexpr int kFusedRouteMaxT = 32;
+
+GemmBuffers gemm_buffers(void* ws, const WsLayout& L, int E) {
+  GemmBuffers g{};
+  g.xq = at<uint8_t>(ws, L.xq);
+  g.xs = at<uint8_t>(ws, L.xs);
+  g.hq = at<uint8_t>(ws, L.hq);
+  g.hs = at<uint8_t>(ws, L.hs);
+  g.item_off0 = at<int32_t>(ws, L.item_off);
+  g.item_off1 = g.item_off0 + (E + 2);
+  return g;
+}
 
 }  // namespace
 
@@ -211,6 +230,7 @@ moe_status_t moe_expert_ffn_mxfp4(const moe_mxfp4_experts_t* experts,
   a.k = shape.k;
   a.has_shared = has_shared;
   a.act_mxfp4 = precision == MOE_ACT_MXFP4;
+  if (rp == MOE_PATH_GEMM) return cuda_status(launch_ffn_gemm(a, gemm_buffers(ws, L, shape.E), s));
   return cuda_status(launch_ffn_gemv(a, s));
 }
 
@@ -291,7 +311,8 @@ moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router, const f
   a.k = shape.k;
   a.has_shared = has_shared;
   a.act_mxfp4 = precision == MOE_ACT_MXFP4;
-  e = launch_ffn_gemv(a, s);
+  e = rp == MOE_PATH_GEMM ? launch_ffn_gemm(a, gemm_buffers(ws, L, shape.E), s)
+                          : launch_ffn_gemv(a, s);
   if (e == cudaSuccess)
     e = launch_combine(a.partial, r.w, shape.T, shape.H, shape.k, has_shared, y, s);
   return cuda_status(e);

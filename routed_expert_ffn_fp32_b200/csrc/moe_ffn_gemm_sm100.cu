@@ -1,0 +1,715 @@
+// Grouped expert FFN on the 5th-generation tensor cores: block-scaled MXFP4
+// x MXFP4 -> float32 (tcgen05.mma kind::mxf4, one E8M0 scale per 32 values
+// on both operands), for prefill-sized batches.
+//
+// The pages run prefill chunks of up to 4K tokens ("ds4-ssd" README,
+// "Validate": 4K prefill chunk cap) and route them through accelerator
+// matmul paths on activations converted for the accelerator ("ds4-ssd"
+// README, "Attribution": GPU dequantisation/packing feeding the ANE routed
+// MLP; intro: NAX matmul2d).  Here the activations are quantised to MXFP4
+// (OCP MX v1.0 rule) so both operands feed the FP4 tensor cores.
+//
+// Per virtual expert v (the activated routed experts in id order, then the
+// shared expert) and per 128-row tile of its weights, one work item computes
+//   D[m, n] = sum_k W[m, k] * A[n, k]      m: weight rows, n: bucket tokens
+// with W on the MMA's M side (128 rows) and the bucket's tokens on its N side
+// (up to kBN per item), so small buckets waste no tensor work on padding.
+// Phase 0: W = gate and up (two accumulators), epilogue h = silu(g) * u,
+// re-quantised to MXFP4 along I.  Phase 1: W = down, epilogue writes the
+// float32 expert outputs into `partial` rows (pair index order).
+//
+// CTA roles (192 threads, one persistent CTA per SM):
+//   warp 0      TMA producer: weight and activation tiles (128-byte swizzle,
+//               no multicast) plus the E8M0 scale bytes, staged by the 32
+//               lanes into the tcgen05 scale-factor atom layout
+//               (byte 16*(r%32) + 4*(r/32%4) + k of a 512-byte atom holds the
+//               scale of row r, K-block k);
+//   warp 1      TMEM allocation; lane 0 issues tcgen05.cp (scales -> TMEM)
+//               and tcgen05.mma, and commits stage / accumulator barriers;
+//   warps 2..5  epilogue: tcgen05.ld of their 32-lane TMEM quarter.
+// Every mbarrier wait is bounded (globaltimer); on expiry the CTA latches
+// MOE_ERR_TIMEOUT in the workspace, drains what it issued and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 128;            // weight rows per item (MMA M)
+constexpr int kBN = 128;            // bucket tokens per item (max MMA N)
+constexpr int kBKB = 128;           // K bytes per stage (256 FP4 values)
+constexpr int kGemmThreads = 192;
+constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
+
+template <int PHASE>
+struct GemmCfg {
+  static constexpr int NPROJ = PHASE == 0 ? 2 : 1;
+  static constexpr int NMB = (kBN + 127) / 128;  // 128-row blocks of B scale factors
+  static constexpr int A_BYTES = kBM * kBKB;     // 16 KB per projection
+  static constexpr int B_BYTES = kBN * kBKB;
+  static constexpr int SFA_BYTES = 2 * 512;      // two K atoms (8 scales) per stage
+  static constexpr int SFB_BYTES = 2 * NMB * 512;
+  static constexpr int STAGE_RAW = NPROJ * A_BYTES + B_BYTES + NPROJ * SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGE = (STAGE_RAW + 1023) / 1024 * 1024;
+  static constexpr int NS = (200 * 1024) / STAGE > 8 ? 8 : (200 * 1024) / STAGE;
+  static constexpr int SMEM = NS * STAGE + 1024 /*barriers*/ + 1024 /*alignment slack*/;
+  // TMEM columns: accumulators, then scale factors
+  static constexpr int ACC_COLS = NPROJ * kBN;
+  static constexpr int SFA_COL = ACC_COLS;                 // NPROJ * 8 columns
+  static constexpr int SFB_COL = ACC_COLS + NPROJ * 8;     // 2 * NMB * 4 columns
+  static constexpr int USED_COLS = SFB_COL + 2 * NMB * 4;
+  static constexpr int TMEM_COLS = USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64
+                                 : USED_COLS <= 128 ? 128 : USED_COLS <= 256 ? 256 : 512;
+  static_assert(USED_COLS <= 512, "TMEM budget");
+};
+
+struct GemmArgs {
+  const int32_t* offsets;
+  const int32_t* entries;
+  const int32_t* plan;
+  const int32_t* item_off;  // [nV + 1] items before virtual expert v
+  const uint8_t* sa[2];     // weight scales of the routed experts [E*ROWS, K/32]
+  const uint8_t* sa_sh[2];  // weight scales of the shared expert [ROWS, K/32]
+  const uint8_t* sb;        // activation scales [rows, K/32]
+  uint8_t* hq;              // phase 0 output codes  [rows, I/2]
+  uint8_t* hs;              // phase 0 output scales [rows, I/32]
+  float* partial;           // phase 1 output [T*k + S*T, H]
+  int* err;
+  int T, H, I, E, k, has_shared;
+};
+
+// ------------------------------------------------------------ primitives ---
+__device__ __forceinline__ uint32_t saddr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; false if it gave up (or another role already did).  Called by
+// one lane; warp_wait() makes the outcome uniform over a warp.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          int* err, int where) {
+  if (mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try(bar, parity)) {
+    if (*abort) return false;
+    if (globaltimer() - t0 > kWaitNs) {
+      *abort = 1;
+      latch_error(err, MOE_ERR_TIMEOUT, where);
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          int* err, int where) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, err, where);
+  return __shfl_sync(kFull, ok, 0) != 0;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+// 32 rows x 16 bytes of scale factors (one 512-byte atom) -> 4 TMEM columns,
+// replicated into the four 32-lane quarters.
+__device__ __forceinline__ void tc_cp_sf(uint32_t tmem, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tmem), "l"(sdesc)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma_mxf4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                            uint32_t accumulate, uint32_t sfa, uint32_t sfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
+  return uint64_t((addr & 0x3FFFFu) >> 4) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+// Descriptor of one scale-factor atom: 32 rows of 16 bytes, no swizzle.
+__device__ __forceinline__ uint64_t desc_sf(uint32_t addr) {
+  return uint64_t((addr & 0x3FFFFu) >> 4) | (uint64_t(128 >> 4) << 32) | (uint64_t(1) << 46);
+}
+// Instruction descriptor: kind::mxf4, E2M1 x E2M1, E8M0 scales, K-major A/B,
+// M = 128, N = n, scale byte pair sf_id for both operands.
+__device__ __forceinline__ uint32_t idesc_mxf4(int n, int sf_id) {
+  return (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (1u << 23) | (uint32_t(kBM >> 4) << 24) |
+         (uint32_t(sf_id) << 29) | (uint32_t(sf_id) << 4);
+}
+
+// 32 columns of this warp's TMEM quarter -> registers
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ------------------------------------------------------------- work items ---
+struct Item {
+  int v;        // virtual expert
+  int e;        // routed expert id, or -1 for the shared expert
+  int mt, nt;   // weight row tile, token tile
+  int row0;     // first activation row of the bucket
+  int R;        // bucket tokens
+  int nvalid;   // tokens of this item
+};
+
+__device__ __forceinline__ Item item_of(const GemmArgs& a, int it, int nA, int nV, int MT) {
+  // virtual expert: last v with item_off[v] <= it
+  int lo = 0, hi = nV - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.item_off[mid] <= it) lo = mid;
+    else hi = mid - 1;
+  }
+  Item r;
+  r.v = lo;
+  const int li = it - a.item_off[lo];
+  const int ntiles = (a.item_off[lo + 1] - a.item_off[lo]) / MT;
+  r.mt = li / ntiles;
+  r.nt = li % ntiles;  // token tiles fastest: neighbours share the weight tile in L2
+  if (lo < nA) {
+    r.e = a.plan[1 + lo];
+    r.row0 = a.offsets[r.e];
+    r.R = a.offsets[r.e + 1] - r.row0;
+  } else {
+    r.e = -1;
+    r.row0 = a.T * a.k;
+    r.R = a.T;
+  }
+  r.nvalid = min(kBN, r.R - r.nt * kBN);
+  return r;
+}
+
+// ------------------------------------------------------------------ kernel ---
+template <int PHASE>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_ffn_gemm(GemmArgs a, const __grid_constant__ CUtensorMap mA0,
+               const __grid_constant__ CUtensorMap mA1, const __grid_constant__ CUtensorMap mS0,
+               const __grid_constant__ CUtensorMap mS1, const __grid_constant__ CUtensorMap mB) {
+  using C = GemmCfg<PHASE>;
+  constexpr int NPROJ = C::NPROJ;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* ctl = smem + C::NS * C::STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctl);
+  uint64_t* empty = full + C::NS;
+  uint64_t* acc_full = empty + C::NS;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(saddr(&full[s]), 1);
+      mbar_init(saddr(&empty[s]), 1);
+    }
+    mbar_init(saddr(acc_full), 1);
+    mbar_init(saddr(acc_empty), 4);
+    mbar_init(saddr(drain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     saddr(tmem_slot)),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  pdl_wait();
+  pdl_trigger();
+
+  const int K = PHASE == 0 ? a.H : a.I;
+  const int ROWS = PHASE == 0 ? a.I : a.H;
+  const int KB = K / 2;        // bytes per row
+  const int NSC = K / 32;      // scale bytes per row
+  const int nks = (KB + kBKB - 1) / kBKB;
+  const int MT = ROWS / kBM;
+  const int nA = a.plan[0];
+  const int nV = nA + (a.has_shared ? 1 : 0);
+  const int n_items = a.item_off[nV];
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t fills = 0;  // bit s: parity of the last fill of stage s
+    uint32_t used = 0;   // bit s: stage s was filled at least once
+    bool ok = true;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const Item w = item_of(a, it, nA, nV, MT);
+      const int arow = (w.e >= 0 ? w.e * ROWS : 0) + w.mt * kBM;
+      const int brow = w.row0 + w.nt * kBN;
+      for (int ks = 0; ks < nks; ++ks) {
+        if (!warp_wait(saddr(&empty[stage]), phase ^ 1u, abort_flag, a.err, 100)) {
+          ok = false;
+          break;
+        }
+        unsigned char* st = smem + stage * C::STAGE;
+        unsigned char* sfa = st + NPROJ * C::A_BYTES + C::B_BYTES;
+        unsigned char* sfb = sfa + NPROJ * C::SFA_BYTES;
+        // scale bytes -> atom layout: K atom a of row r at a*512*mb + 16*(r%32) + 4*(r/32%4)
+        const int sc0 = ks * 8;  // first scale byte of this stage
+#pragma unroll
+        for (int p = 0; p < NPROJ; ++p) {
+          const uint8_t* src = (w.e >= 0 ? a.sa[p] : a.sa_sh[p]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int r = lane + 32 * j;
+            const uint8_t* rowp = src + size_t(arow + r) * NSC;
+#pragma unroll
+            for (int at = 0; at < 2; ++at) {
+              const int c = sc0 + 4 * at;
+              const uint32_t word =
+                  c + 4 <= NSC ? *reinterpret_cast<const uint32_t*>(rowp + c) : 0x7f7f7f7fu;
+              *reinterpret_cast<uint32_t*>(sfa + p * C::SFA_BYTES + at * 512 + 16 * (r % 32) +
+                                           4 * (r / 32)) = word;
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < C::NMB * 4; ++j) {
+          const int n = lane + 32 * j;
+          const uint8_t* rowp = a.sb + size_t(brow + n) * NSC;
+#pragma unroll
+          for (int at = 0; at < 2; ++at) {
+            const int c = sc0 + 4 * at;
+            const uint32_t word = (n < w.nvalid && c + 4 <= NSC)
+                                      ? *reinterpret_cast<const uint32_t*>(rowp + c)
+                                      : 0x7f7f7f7fu;
+            *reinterpret_cast<uint32_t*>(sfb + at * C::NMB * 512 + (n / 128) * 512 +
+                                         16 * (n % 32) + 4 * ((n / 32) % 4)) = word;
+          }
+        }
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t fb = saddr(&full[stage]);
+          mbar_expect_tx(fb, NPROJ * C::A_BYTES + C::B_BYTES);
+          const CUtensorMap* ma0 = w.e >= 0 ? &mA0 : &mS0;
+          tma_load_2d(saddr(st), ma0, ks * kBKB, arow, fb);
+          if constexpr (NPROJ == 2) {
+            const CUtensorMap* ma1 = w.e >= 0 ? &mA1 : &mS1;
+            tma_load_2d(saddr(st + C::A_BYTES), ma1, ks * kBKB, arow, fb);
+          }
+          tma_load_2d(saddr(st + NPROJ * C::A_BYTES), &mB, ks * kBKB, brow, fb);
+        }
+        __syncwarp();
+        fills ^= 1u << stage;  // parity of this fill's phase = bit after toggle ^ 1
+        used |= 1u << stage;
+        if (++stage == C::NS) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // after a give-up, let every tile this warp requested land (bounded)
+    if (*abort_flag && lane == 0) {
+      for (int s = 0; s < C::NS; ++s) {
+        if (!((used >> s) & 1u)) continue;
+        const uint32_t last_parity = ((fills >> s) & 1u) ^ 1u;
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try(saddr(&full[s]), last_parity) && globaltimer() - t0 < 100000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      const uint32_t tsfa = tmem + C::SFA_COL;
+      const uint32_t tsfb = tmem + C::SFB_COL;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const Item w = item_of(a, it, nA, nV, MT);
+        const int n_mma = ((w.nvalid + 7) / 8) * 8;
+        if (!mbar_wait(saddr(acc_empty), acc_phase ^ 1u, abort_flag, a.err, 200)) break;
+        tc_fence_after();
+        for (int ks = 0; ks < nks; ++ks) {
+          if (!mbar_wait(saddr(&full[stage]), phase, abort_flag, a.err, 201)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          unsigned char* st = smem + stage * C::STAGE;
+          unsigned char* sfa = st + NPROJ * C::A_BYTES + C::B_BYTES;
+          unsigned char* sfb = sfa + NPROJ * C::SFA_BYTES;
+#pragma unroll
+          for (int p = 0; p < NPROJ; ++p)
+#pragma unroll
+            for (int at = 0; at < 2; ++at)
+              tc_cp_sf(tsfa + p * 8 + at * 4, desc_sf(saddr(sfa + p * C::SFA_BYTES + at * 512)));
+#pragma unroll
+          for (int at = 0; at < 2; ++at)
+#pragma unroll
+            for (int mb = 0; mb < C::NMB; ++mb)
+              tc_cp_sf(tsfb + (at * C::NMB + mb) * 4,
+                       desc_sf(saddr(sfb + at * C::NMB * 512 + mb * 512)));
+          const int kb_n = min(4, (KB - ks * kBKB) / 32);  // 64-value K blocks in this stage
+          for (int kb = 0; kb < kb_n; ++kb) {
+            const uint32_t id = idesc_mxf4(n_mma, (kb & 1) * 2);
+            const uint64_t bdesc = desc_sw128(saddr(st + NPROJ * C::A_BYTES) + kb * 32);
+#pragma unroll
+            for (int p = 0; p < NPROJ; ++p) {
+              const uint64_t adesc = desc_sw128(saddr(st + p * C::A_BYTES) + kb * 32);
+              tc_mma_mxf4(tmem + p * kBN, adesc, bdesc, id, (ks | kb) != 0,
+                          tsfa + p * 8 + (kb >> 1) * 4, tsfb + (kb >> 1) * C::NMB * 4);
+            }
+          }
+          tc_commit(saddr(&empty[stage]));
+          if (++stage == C::NS) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(saddr(acc_full));
+        acc_phase ^= 1u;
+      }
+      if (!ok || *abort_flag) {
+        // give-up path: let issued MMAs finish before TMEM is released
+        tc_commit(saddr(drain));
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try(saddr(drain), 0) && globaltimer() - t0 < 200000000ull) {
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    uint32_t acc_phase = 0;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+      const Item w = item_of(a, it, nA, nV, MT);
+      if (!warp_wait(saddr(acc_full), acc_phase, abort_flag, a.err, 300)) break;
+      tc_fence_after();
+      const int wrow = w.mt * kBM + 32 * q + lane;  // weight row of this lane
+      for (int c0 = 0; c0 < w.nvalid; c0 += 32) {
+        const uint32_t taddr = tmem + (uint32_t(32 * q) << 16) + c0;
+        if constexpr (PHASE == 0) {
+          float g[32], u[32];
+          tmem_ld32(taddr, g);
+          tmem_ld32(taddr + kBN, u);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int n = c0 + j;
+            const float h = g[j] / (1.f + expf(-g[j])) * u[j];
+            float amax = fabsf(h);
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1)
+              amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
+            const int X = mx_scale_exponent(amax);
+            const float hn = __shfl_down_sync(kFull, h, 1);
+            if (n < w.nvalid) {
+              const size_t orow = size_t(w.row0 + w.nt * kBN + n);
+              if ((lane & 1) == 0) {
+                const float inv = exp2i(-X);
+                a.hq[orow * (a.I / 2) + (w.mt * kBM + 32 * q) / 2 + lane / 2] =
+                    uint8_t(f32x2_to_e2m1x2(h * inv, hn * inv));
+              }
+              if (lane == 0) a.hs[orow * (a.I / 32) + (w.mt * kBM + 32 * q) / 32] = uint8_t(X + 127);
+            }
+          }
+        } else {
+          float o[32];
+          tmem_ld32(taddr, o);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int n = c0 + j;
+            if (n < w.nvalid) {
+              const int r = w.nt * kBN + n;
+              const int prow = w.e >= 0 ? a.entries[w.row0 + r] : a.T * a.k + r;
+              a.partial[size_t(prow) * a.H + wrow] = o[j];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(saddr(acc_empty));
+      acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------- activation gather ---
+// Row r < T*k of the gathered operand is token entries[r] / k (bucket order);
+// rows T*k + t are token t (shared expert).  One warp per row.
+__global__ void __launch_bounds__(256) k_act_gather(const uint16_t* x, const int32_t* entries,
+                                                    int T, int H, int k, int rows, uint8_t* q,
+                                                    uint8_t* s) {
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 8 + warp;
+  if (r >= rows) return;
+  const int tok = r < T * k ? entries[r] / k : r - T * k;
+  const uint16_t* src = x + size_t(tok) * H;
+  const int nb = H / 32;
+  for (int b = lane; b < nb; b += 32) {
+    const uint4* p = reinterpret_cast<const uint4*>(src + size_t(b) * 32);
+    float f[32];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 v = __ldg(p + j);
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        f[8 * j + 2 * i] = bf16_bits_to_f32(wv[i] & 0xffffu);
+        f[8 * j + 2 * i + 1] = bf16_bits_to_f32(wv[i] >> 16);
+      }
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    const int X = mx_scale_exponent(amax);
+    const float inv = exp2i(-X);
+    uint32_t word[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t acc = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        acc |= f32x2_to_e2m1x2(f[8 * j + 2 * i] * inv, f[8 * j + 2 * i + 1] * inv) << (8 * i);
+      word[j] = acc;
+    }
+    *reinterpret_cast<uint4*>(q + size_t(r) * (H / 2) + size_t(b) * 16) =
+        make_uint4(word[0], word[1], word[2], word[3]);
+    s[size_t(r) * nb + b] = uint8_t(X + 127);
+  }
+}
+
+// ------------------------------------------------------- item prefix sums ---
+// item_off[p][v] = sum_{v' < v} MT_p * ceil(R_v' / kBN) for both phases.
+__global__ void __launch_bounds__(1024) k_gemm_plan(const int32_t* offsets, const int32_t* plan,
+                                                    int T, int k, int has_shared, int MT0, int MT1,
+                                                    int32_t* item_off0, int32_t* item_off1) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int tiles[kMaxExperts + 2];
+  __shared__ int wsum[33];
+  const int nA = plan[0];
+  const int nV = nA + (has_shared ? 1 : 0);
+  for (int v = threadIdx.x; v < nV; v += blockDim.x) {
+    int R;
+    if (v < nA) {
+      const int e = plan[1 + v];
+      R = offsets[e + 1] - offsets[e];
+    } else {
+      R = T;
+    }
+    tiles[v] = (R + kBN - 1) / kBN;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    // one warp: running prefix in chunks of 32
+    int run = 0;
+    for (int base = 0; base < nV; base += 32) {
+      const int v = base + threadIdx.x;
+      const int t = v < nV ? tiles[v] : 0;
+      int incl = t;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(kFull, incl, off);
+        if ((int)threadIdx.x >= off) incl += y;
+      }
+      if (v < nV) {
+        item_off0[v] = (run + incl - t) * MT0;
+        item_off1[v] = (run + incl - t) * MT1;
+      }
+      run += __shfl_sync(kFull, incl, 31);
+    }
+    if (threadIdx.x == 0) {
+      item_off0[nV] = run * MT0;
+      item_off1[nV] = run * MT1;
+    }
+  }
+  (void)wsum;
+}
+
+// --------------------------------------------------------------- host side ---
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    cudaDriverEntryPointQueryResult q{};
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D map of a [rows, row_bytes] uint8 matrix, boxes of box_rows x 128 bytes.
+bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
+              uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {uint32_t(kBKB), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int PHASE>
+cudaError_t launch_gemm_phase(const GemmArgs& g, const CUtensorMap& a0, const CUtensorMap& a1,
+                              const CUtensorMap& s0, const CUtensorMap& s1, const CUtensorMap& b,
+                              cudaStream_t st) {
+  using C = GemmCfg<PHASE>;
+  auto kern = k_ffn_gemm<PHASE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(device_info().sm_count), dim3(kGemmThreads), size_t(C::SMEM), st, g,
+                    a0, a1, s0, s1, b);
+}
+
+}  // namespace
+
+bool gemm_supported(const moe_shape_t& s) {
+  return s.H % 256 == 0 && s.I % 128 == 0 && encode_fn() != nullptr;
+}
+
+cudaError_t launch_ffn_gemm(const FfnArgs& a, const GemmBuffers& gb, cudaStream_t st) {
+  const int rows = a.T * a.k + (a.has_shared ? a.T : 0);
+  cudaError_t e = launch_pdl(k_act_gather, dim3((rows + 7) / 8), dim3(256), 0, st, a.x, a.entries,
+                             a.T, a.H, a.k, rows, gb.xq, gb.xs);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(k_gemm_plan, dim3(1), dim3(1024), 0, st, a.offsets, a.plan, a.T, a.k,
+                 a.has_shared, a.I / kBM, a.H / kBM, gb.item_off0, gb.item_off1);
+  if (e != cudaSuccess) return e;
+
+  CUtensorMap g0, g1, sg0, sg1, bx, d0, sd0, bh;
+  const uint64_t HB = a.H / 2, IB = a.I / 2;
+  bool ok = make_map(&g0, a.ex.gq, HB, uint64_t(a.E) * a.I, kBM) &&
+            make_map(&g1, a.ex.uq, HB, uint64_t(a.E) * a.I, kBM) &&
+            make_map(&bx, gb.xq, HB, rows, kBN) &&
+            make_map(&d0, a.ex.dq, IB, uint64_t(a.E) * a.H, kBM) &&
+            make_map(&bh, gb.hq, IB, rows, kBN);
+  if (a.has_shared) {
+    ok = ok && make_map(&sg0, a.sh.gq, HB, a.I, kBM) && make_map(&sg1, a.sh.uq, HB, a.I, kBM) &&
+         make_map(&sd0, a.sh.dq, IB, a.H, kBM);
+  } else {
+    sg0 = g0;
+    sg1 = g1;
+    sd0 = d0;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+
+  GemmArgs g{};
+  g.offsets = a.offsets;
+  g.entries = a.entries;
+  g.plan = a.plan;
+  g.err = a.err;
+  g.T = a.T;
+  g.H = a.H;
+  g.I = a.I;
+  g.E = a.E;
+  g.k = a.k;
+  g.has_shared = a.has_shared;
+  // phase 0: gate/up, SwiGLU, MXFP4 h
+  g.item_off = gb.item_off0;
+  g.sa[0] = a.ex.gs;
+  g.sa[1] = a.ex.us;
+  g.sa_sh[0] = a.has_shared ? a.sh.gs : a.ex.gs;
+  g.sa_sh[1] = a.has_shared ? a.sh.us : a.ex.us;
+  g.sb = gb.xs;
+  g.hq = gb.hq;
+  g.hs = gb.hs;
+  e = launch_gemm_phase<0>(g, g0, g1, sg0, sg1, bx, st);
+  if (e != cudaSuccess) return e;
+  // phase 1: down
+  g.item_off = gb.item_off1;
+  g.sa[0] = a.ex.ds;
+  g.sa[1] = a.ex.ds;
+  g.sa_sh[0] = a.has_shared ? a.sh.ds : a.ex.ds;
+  g.sa_sh[1] = g.sa_sh[0];
+  g.sb = gb.hs;
+  g.partial = a.partial;
+  return launch_gemm_phase<1>(g, d0, d0, sd0, sd0, bh, st);
+}
+
+}  // namespace moe

@@ -32,8 +32,10 @@ struct WsLayout {
   size_t plan;      // i32 [E + 2]: [0] active experts, [1..] their ids (ascending)
   size_t h;         // f32 [T*k + S*T, I]   SwiGLU output rows (by pair index)
   size_t partial;   // f32 [T*k + S*T, H]   expert output rows (by pair index)
-  size_t aq;        // u8  [T*k + S*T, max(H,I)/2]  MXFP4 activation codes (GEMM path)
-  size_t as;        // u8  [T*k + S*T, max(H,I)/32] MXFP4 activation scales (GEMM path)
+  // tensor-core path only
+  size_t xq, xs;    // u8 [rows, H/2], [rows, H/32]  MXFP4 token rows, bucket order
+  size_t hq, hs;    // u8 [rows, I/2], [rows, I/32]  MXFP4 SwiGLU rows, bucket order
+  size_t item_off;  // i32 [2][E + 2]  work-item prefix sums of the two GEMM phases
   size_t total;
 };
 
@@ -57,9 +59,15 @@ inline WsLayout ws_layout(const moe_shape_t& s, int has_shared, int gemm) {
   L.plan = take((E + 2) * 4);
   L.h = take(rows * I * 4);
   L.partial = take(rows * H * 4);
-  const size_t KM = H > I ? H : I;
-  L.aq = gemm ? take(rows * KM / 2) : o;
-  L.as = gemm ? take(rows * KM / 32) : o;
+  if (gemm) {
+    L.xq = take(rows * H / 2);
+    L.xs = take(rows * H / 32);
+    L.hq = take(rows * I / 2);
+    L.hs = take(rows * I / 32);
+    L.item_off = take(2 * (E + 2) * 4);
+  } else {
+    L.xq = L.xs = L.hq = L.hs = L.item_off = o;
+  }
   L.total = o;
   return L;
 }
@@ -231,6 +239,17 @@ cudaError_t launch_bucket(const RouteArgs& a, cudaStream_t st);
 cudaError_t launch_plan(const RouteArgs& a, cudaStream_t st);
 
 cudaError_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t st);
+
+struct GemmBuffers {
+  uint8_t* xq;
+  uint8_t* xs;
+  uint8_t* hq;
+  uint8_t* hs;
+  int32_t* item_off0;
+  int32_t* item_off1;
+};
+bool gemm_supported(const moe_shape_t& s);
+cudaError_t launch_ffn_gemm(const FfnArgs& a, const GemmBuffers& gb, cudaStream_t st);
 cudaError_t launch_combine(const float* partial, const float* w, int T, int H, int k,
                            int has_shared, uint16_t* y, cudaStream_t st);
 cudaError_t launch_act_quant(const float* in, int rows, int K, uint8_t* q, uint8_t* s,
