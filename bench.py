@@ -41,11 +41,21 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--T", type=int, default=DEFAULT_T)
     ap.add_argument("--layers", type=int, default=8)
+    ap.add_argument("--precision", choices=["exact", "mxfp4"], default="exact",
+                    help="activation precision of the expert projections")
+    ap.add_argument("--path", choices=["auto", "gemv", "gemm"], default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
     a = ap.parse_args()
     a.warmup = max(3, a.warmup)
     return a
+
+
+def _consts(args):
+    from routed_expert_ffn_fp32_b200 import moe
+    prec = moe.MOE_ACT_MXFP4 if args.precision == "mxfp4" else moe.MOE_ACT_EXACT
+    path = {"auto": moe.MOE_PATH_AUTO, "gemv": moe.MOE_PATH_GEMV, "gemm": moe.MOE_PATH_GEMM}[args.path]
+    return prec, path
 
 
 # ---------------------------------------------------------------- clocks ---
@@ -137,6 +147,7 @@ def run_ours(args, rank, world, local_rank):
     moe.load_library()
     cfg = workload(args.workload, args.T)
     T, NL = cfg.T, args.layers
+    PREC, PATH = _consts(args)
     L = synth.layer(cfg, seed=0)
     W_r, bias = L["W_r"], L["bias"]
     ex0 = moe.Experts.from_numpy(L["experts"], dev)
@@ -156,15 +167,15 @@ def run_ours(args, rank, world, local_rank):
     xs = [torch.from_numpy(a.view(np.int16)).to(dev) for a in xs_np]
     shape = moe.shape_of(T, cfg.H, cfg.I, cfg.E, cfg.k)
     stream = torch.cuda.Stream(dev)
-    ws = moe.make_workspace(shape, moe.MOE_PATH_AUTO, moe.MOE_ACT_EXACT, cfg.shared, dev, stream)
+    ws = moe.make_workspace(shape, PATH, PREC, cfg.shared, dev, stream)
     y = torch.empty((T, cfg.H), dtype=torch.int16, device=dev)
     idx = torch.empty((T, cfg.k), dtype=torch.int32, device=dev)
     wts = torch.empty((T, cfg.k), dtype=torch.float32, device=dev)
 
     def call(i, st):
         ex, sh = layers[i % NL]
-        moe.moe_layer_forward(xs[i % NX], Wd, bd, ex, sh, shape, y, ws, moe.MOE_PATH_AUTO,
-                              moe.MOE_ACT_EXACT, idx, wts, stream=st)
+        moe.moe_layer_forward(xs[i % NX], Wd, bd, ex, sh, shape, y, ws, PATH, PREC, idx, wts,
+                              stream=st)
 
     # one graph per (layer copy, batch) pair in the cycle
     ncyc = int(np.lcm(NL, NX))
@@ -247,7 +258,7 @@ def run_ours(args, rank, world, local_rank):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 moe.moe_expert_ffn_mxfp4(ex, sh, xs[i % NX], o_i, e_i, shape, partial, ws,
-                                         moe.MOE_PATH_AUTO, moe.MOE_ACT_EXACT, stream=stream)
+                                         PATH, PREC, stream=stream)
             ffn_graphs.append((g, o_i, e_i))
         for i in range(args.warmup):
             ffn_graphs[i % ncyc][0].replay()
@@ -264,11 +275,27 @@ def run_ours(args, rank, world, local_rank):
     ffn_b = float(np.mean([ffn_bytes[i % ncyc] for i in range(nrep)]))
     peaks = load_peaks()
     achieved = ffn_b / (ffn_ms / 1e3) / 1e9
+    flops = 6.0 * cfg.H * cfg.I * T * (cfg.k + (1 if cfg.shared else 0))
+    tflops = flops / (ffn_ms / 1e3) / 1e12
+    uses_tc = PREC == moe.MOE_ACT_MXFP4 and (
+        PATH == moe.MOE_PATH_GEMM or (PATH == moe.MOE_PATH_AUTO and T * cfg.k >= 512))
+    fp4_peak = peaks["bf16_tflops"] * 4.0  # dense FP4 = 4 x dense bf16 (nominal ratio)
+    t_hbm = ffn_b / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (fp4_peak * 1e12)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": None, "kernel": "expert FFN (gate/up + SwiGLU, down)",
                 "peak_source": peaks["source"], "bytes_per_launch": int(ffn_b),
                 "launch_ms": round(ffn_ms, 5)}
+    if uses_tc:
+        roofline["kernel"] = "expert FFN on tcgen05 kind::mxf4 (gate/up + SwiGLU + requant, down)"
+        roofline["tensor"] = {
+            "achieved_tflops": round(tflops, 1), "fp4_peak_tflops": round(fp4_peak, 1),
+            "frac_of_fp4_peak": round(tflops / fp4_peak, 4),
+            "fp4_peak_source": "measured bf16 burst x 4 (nominal dense FP4/bf16 ratio)",
+            "flops_per_launch": flops,
+            "attainable_frac": round(max(t_hbm, t_tc) / (ffn_ms / 1e3), 4),
+            "bound_by": "hbm" if t_hbm >= t_tc else "tensor"}
     layer_gbs = bytes_per_call / (ms_local / 1e3) / 1e9
 
     # ---- end to end through the C ABI with host buffers ------------------------
@@ -280,7 +307,7 @@ def run_ours(args, rank, world, local_rank):
         for i in range(args.warmup):
             xd.copy_(xh[i % NX], non_blocking=True)
             ex, sh = layers[i % NL]
-            moe.moe_layer_forward(xd, Wd, bd, ex, sh, shape, y, ws, stream=stream)
+            moe.moe_layer_forward(xd, Wd, bd, ex, sh, shape, y, ws, PATH, PREC, stream=stream)
             yh.copy_(y, non_blocking=True)
         stream.synchronize()
         g0 = torch.cuda.Event(enable_timing=True)
@@ -289,7 +316,7 @@ def run_ours(args, rank, world, local_rank):
         for i in range(n_e2e):
             xd.copy_(xh[i % NX], non_blocking=True)
             ex, sh = layers[i % NL]
-            moe.moe_layer_forward(xd, Wd, bd, ex, sh, shape, y, ws, stream=stream)
+            moe.moe_layer_forward(xd, Wd, bd, ex, sh, shape, y, ws, PATH, PREC, stream=stream)
             yh.copy_(y, non_blocking=True)
         g1.record(stream)
         stream.synchronize()
@@ -298,16 +325,20 @@ def run_ours(args, rank, world, local_rank):
            "h2d_bytes_per_step": T * cfg.H * 2, "d2h_bytes_per_step": T * cfg.H * 2,
            "ms_per_step": round(e2e_ms, 5), "api": "moe_layer_forward (eager, ctypes)"}
 
-    launches_per_step = 4 if T <= 32 else 6
+    # route (fused for T <= 32) + gate/up + down + combine; the tensor-core path
+    # adds the activation gather and the work-item plan
+    launches_per_step = (4 if T <= 32 else 6) + (2 if uses_tc else 0)
     clocks = sampler.summary(h0, h1)
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic",
+        "dtype": "f32" if PREC == moe.MOE_ACT_EXACT else "mxfp4 x mxfp4 -> f32",
+        "data": "synthetic",
         "config": {"workload": cfg.name, "T": T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
                    "shared": cfg.shared, "weights": "MXFP4 (E2M1 + E8M0 per 32)",
-                   "activations": "bf16", "accumulate": "f32",
+                   "activations": "bf16" if PREC == moe.MOE_ACT_EXACT else "MXFP4 (quantised)",
+                   "accumulate": "f32", "path": args.path,
                    "layer_copies": NL,
                    "l2": f"inputs larger than L2: {NL} layer copies "
                          f"({NL * cfg.E * expert_bytes(cfg) / 1e9:.2f} GB) cycled",
