@@ -182,6 +182,27 @@ MOE_API moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router,
                                int32_t* topk_idx_out, float* topk_w_out,
                                void* ws, size_t ws_bytes, void* stream);
 
+/* The whole layer like moe_layer_forward (CUDA-core GEMV path) but with no
+ * workspace argument and no allocation of any kind.  The pages have no
+ * counterpart: this serves callers that may not allocate device memory (a host
+ * application that owns every allocation through its own pool, a real-time
+ * loop where cudaMalloc/cudaFree could synchronise the device, plug-in code
+ * that only receives its input and output tensors).  Scratch is a fixed
+ * 16 MiB array inside the library's device image, held on every GPU that loads
+ * the library until the process exits; a shape whose moe_workspace_bytes(...,
+ * MOE_PATH_GEMV, ...) exceeds it returns MOE_ERR_WORKSPACE.  The first call on
+ * a device looks up the array's device address (make it before any stream
+ * capture).  Every call reuses the same array: calls that overlap on the GPU
+ * race and must be ordered on one stream.  Inputs and outputs as for
+ * moe_layer_forward; topk_idx_out / topk_w_out may be NULL. */
+MOE_API moe_status_t moe_layer_forward_static(const uint16_t* x, const float* w_router,
+                                              const float* bias,
+                                              const moe_mxfp4_experts_t* experts,
+                                              const moe_mxfp4_experts_t* shared,
+                                              moe_shape_t shape, int32_t precision,
+                                              uint16_t* y, int32_t* topk_idx_out,
+                                              float* topk_w_out, void* stream);
+
 /* Quantise rows [rows, K] float32 to MXFP4 (codes [rows, K/2], scales
  * [rows, K/32]) with the MOE_ACT_MXFP4 rule above; K % 32 == 0. */
 MOE_API moe_status_t moe_act_quant_mxfp4(const float* in, int32_t rows, int32_t K,

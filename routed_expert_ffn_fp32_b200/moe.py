@@ -37,6 +37,7 @@ EXPORTS = (
     "moe_workspace_bytes", "moe_workspace_init", "moe_route_topk", "moe_bucket",
     "moe_expert_ffn_mxfp4", "moe_combine", "moe_layer_forward", "moe_act_quant_mxfp4",
     "moe_decode_mxfp4", "moe_get_error", "moe_status_string", "moe_version",
+    "moe_layer_forward_static",
 )
 
 
@@ -83,6 +84,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "moe_expert_ffn_mxfp4": (i32, [ex, ex, vp, vp, vp, shape, i32, i32, vp, vp, sz, vp]),
         "moe_combine": (i32, [vp, vp, shape, i32, vp, vp]),
         "moe_layer_forward": (i32, [vp, vp, vp, ex, ex, shape, i32, i32, vp, vp, vp, vp, sz, vp]),
+        "moe_layer_forward_static": (i32, [vp, vp, vp, ex, ex, shape, i32, vp, vp, vp, vp]),
         "moe_act_quant_mxfp4": (i32, [vp, i32, i32, vp, vp, vp]),
         "moe_decode_mxfp4": (i32, [vp, vp, i32, i32, vp, vp]),
         "moe_get_error": (i32, [vp, vp]),
@@ -215,6 +217,16 @@ def moe_layer_forward(x, w_router, bias, experts: Experts, shared, shape, y, ws,
                                             _ex(shared), shape, path, precision, _p(y),
                                             _p(topk_idx), _p(topk_w), _p(ws), ws.numel(),
                                             _s(stream)), "moe_layer_forward")
+
+
+def moe_layer_forward_static(x, w_router, bias, experts: Experts, shared, shape, y,
+                             precision=MOE_ACT_EXACT, topk_idx=None, topk_w=None, stream=None):
+    """moe_layer_forward without a workspace: the library's own fixed scratch
+    array stands in for it (for callers that may not allocate)."""
+    _check(load_library().moe_layer_forward_static(_p(x), _p(w_router), _p(bias), _ex(experts),
+                                                   _ex(shared), shape, precision, _p(y),
+                                                   _p(topk_idx), _p(topk_w), _s(stream)),
+           "moe_layer_forward_static")
 
 
 def moe_act_quant_mxfp4(inp, q_out, s_out, stream=None):
