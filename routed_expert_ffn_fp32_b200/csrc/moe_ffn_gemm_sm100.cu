@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
-      mbar_init(saddr(&full[s]), 1);
+      mbar_init(saddr(&full[s]), 2);
       mbar_init(saddr(&empty[s]), 1);
     }
     mbar_init(saddr(acc_full), 1);
@@ -301,76 +301,113 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Stages are numbered g = 0.. over this CTA's items (nks stages each).
+    // The scale words of stage g+1 are loaded into registers while stage g
+    // waits for its slot, so their global latency overlaps the pipeline; the
+    // tile TMAs are issued before the scales are written, and the stage's full
+    // barrier takes two arrivals (TMA transaction + scales staged).
+    constexpr int NB_ROWS = C::NMB * 4;  // 32-row groups of B scale rows
     int stage = 0;
     uint32_t phase = 0;
     uint32_t fills = 0;  // bit s: parity of the last fill of stage s
     uint32_t used = 0;   // bit s: stage s was filled at least once
     bool ok = true;
-    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-      const Item w = item_of(a, it, nA, nV, MT);
-      const int arow = (w.e >= 0 ? w.e * ROWS : 0) + w.mt * kBM;
-      const int brow = w.row0 + w.nt * kBN;
-      for (int ks = 0; ks < nks; ++ks) {
-        if (!warp_wait(saddr(&empty[stage]), phase ^ 1u, abort_flag, a.err, 100)) {
-          ok = false;
-          break;
-        }
-        unsigned char* st = smem + stage * C::STAGE;
-        unsigned char* sfa = st + NPROJ * C::A_BYTES + C::B_BYTES;
-        unsigned char* sfb = sfa + NPROJ * C::SFA_BYTES;
-        // scale bytes -> atom layout: K atom a of row r at a*512*mb + 16*(r%32) + 4*(r/32%4)
-        const int sc0 = ks * 8;  // first scale byte of this stage
+    const int my_items = n_items > int(blockIdx.x) ? (n_items - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
+    const int total = my_items * nks;
+    Item wn{};
+    int arow_n = 0, brow_n = 0, ks_n = 0;
+    uint32_t sa_n[NPROJ][4][2], sb_n[NB_ROWS][2];
+    auto prepare = [&](int g) {
+      ks_n = g % nks;
+      if (ks_n == 0) {
+        wn = item_of(a, int(blockIdx.x) + (g / nks) * int(gridDim.x), nA, nV, MT);
+        arow_n = (wn.e >= 0 ? wn.e * ROWS : 0) + wn.mt * kBM;
+        brow_n = wn.row0 + wn.nt * kBN;
+      }
+      const int sc0 = ks_n * 8;  // first scale byte of the stage
 #pragma unroll
-        for (int p = 0; p < NPROJ; ++p) {
-          const uint8_t* src = (w.e >= 0 ? a.sa[p] : a.sa_sh[p]);
+      for (int p = 0; p < NPROJ; ++p) {
+        const uint8_t* src = (wn.e >= 0 ? a.sa[p] : a.sa_sh[p]);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int r = lane + 32 * j;
-            const uint8_t* rowp = src + size_t(arow + r) * NSC;
-#pragma unroll
-            for (int at = 0; at < 2; ++at) {
-              const int c = sc0 + 4 * at;
-              const uint32_t word =
-                  c + 4 <= NSC ? *reinterpret_cast<const uint32_t*>(rowp + c) : 0x7f7f7f7fu;
-              *reinterpret_cast<uint32_t*>(sfa + p * C::SFA_BYTES + at * 512 + 16 * (r % 32) +
-                                           4 * (r / 32)) = word;
-            }
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < C::NMB * 4; ++j) {
-          const int n = lane + 32 * j;
-          const uint8_t* rowp = a.sb + size_t(brow + n) * NSC;
+        for (int j = 0; j < 4; ++j) {
+          const uint8_t* rowp = src + size_t(arow_n + lane + 32 * j) * NSC;
 #pragma unroll
           for (int at = 0; at < 2; ++at) {
             const int c = sc0 + 4 * at;
-            const uint32_t word = (n < w.nvalid && c + 4 <= NSC)
-                                      ? *reinterpret_cast<const uint32_t*>(rowp + c)
-                                      : 0x7f7f7f7fu;
-            *reinterpret_cast<uint32_t*>(sfb + at * C::NMB * 512 + (n / 128) * 512 +
-                                         16 * (n % 32) + 4 * ((n / 32) % 4)) = word;
+            sa_n[p][j][at] = c + 4 <= NSC ? __ldg(reinterpret_cast<const uint32_t*>(rowp + c))
+                                          : 0x7f7f7f7fu;
           }
         }
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) {
-          const uint32_t fb = saddr(&full[stage]);
-          mbar_expect_tx(fb, NPROJ * C::A_BYTES + C::B_BYTES);
-          const CUtensorMap* ma0 = w.e >= 0 ? &mA0 : &mS0;
-          tma_load_2d(saddr(st), ma0, ks * kBKB, arow, fb);
-          if constexpr (NPROJ == 2) {
-            const CUtensorMap* ma1 = w.e >= 0 ? &mA1 : &mS1;
-            tma_load_2d(saddr(st + C::A_BYTES), ma1, ks * kBKB, arow, fb);
-          }
-          tma_load_2d(saddr(st + NPROJ * C::A_BYTES), &mB, ks * kBKB, brow, fb);
+      }
+#pragma unroll
+      for (int j = 0; j < NB_ROWS; ++j) {
+        const int n = lane + 32 * j;
+        const uint8_t* rowp = a.sb + size_t(brow_n + n) * NSC;
+#pragma unroll
+        for (int at = 0; at < 2; ++at) {
+          const int c = sc0 + 4 * at;
+          sb_n[j][at] = (n < wn.nvalid && c + 4 <= NSC)
+                            ? __ldcg(reinterpret_cast<const uint32_t*>(rowp + c))
+                            : 0x7f7f7f7fu;
         }
-        __syncwarp();
-        fills ^= 1u << stage;  // parity of this fill's phase = bit after toggle ^ 1
-        used |= 1u << stage;
-        if (++stage == C::NS) {
-          stage = 0;
-          phase ^= 1u;
+      }
+    };
+    if (total > 0) prepare(0);
+    for (int g = 0; g < total && ok; ++g) {
+      const int ks = ks_n, arow = arow_n, brow = brow_n;
+      const bool routed = wn.e >= 0;
+      uint32_t sa[NPROJ][4][2], sb[NB_ROWS][2];
+#pragma unroll
+      for (int p = 0; p < NPROJ; ++p)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          sa[p][j][0] = sa_n[p][j][0];
+          sa[p][j][1] = sa_n[p][j][1];
         }
+#pragma unroll
+      for (int j = 0; j < NB_ROWS; ++j) {
+        sb[j][0] = sb_n[j][0];
+        sb[j][1] = sb_n[j][1];
+      }
+      if (g + 1 < total) prepare(g + 1);
+      if (!warp_wait(saddr(&empty[stage]), phase ^ 1u, abort_flag, a.err, 100)) {
+        ok = false;
+        break;
+      }
+      unsigned char* st = smem + stage * C::STAGE;
+      unsigned char* sfa = st + NPROJ * C::A_BYTES + C::B_BYTES;
+      unsigned char* sfb = sfa + NPROJ * C::SFA_BYTES;
+      const uint32_t fb = saddr(&full[stage]);
+      if (lane == 0) {
+        mbar_expect_tx(fb, NPROJ * C::A_BYTES + C::B_BYTES);
+        tma_load_2d(saddr(st), routed ? &mA0 : &mS0, ks * kBKB, arow, fb);
+        if constexpr (NPROJ == 2)
+          tma_load_2d(saddr(st + C::A_BYTES), routed ? &mA1 : &mS1, ks * kBKB, arow, fb);
+        tma_load_2d(saddr(st + NPROJ * C::A_BYTES), &mB, ks * kBKB, brow, fb);
+      }
+      // scale words -> atom layout: K atom `at` of row r at at*512 + 16*(r%32) + 4*(r/32%4)
+#pragma unroll
+      for (int p = 0; p < NPROJ; ++p)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int at = 0; at < 2; ++at)
+            *reinterpret_cast<uint32_t*>(sfa + p * C::SFA_BYTES + at * 512 + 16 * lane + 4 * j) =
+                sa[p][j][at];
+#pragma unroll
+      for (int j = 0; j < NB_ROWS; ++j)
+#pragma unroll
+        for (int at = 0; at < 2; ++at)
+          *reinterpret_cast<uint32_t*>(sfb + at * C::NMB * 512 + (j / 4) * 512 + 16 * lane +
+                                       4 * (j % 4)) = sb[j][at];
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(fb);
+      fills ^= 1u << stage;  // parity of this fill's phase = bit after toggle ^ 1
+      used |= 1u << stage;
+      if (++stage == C::NS) {
+        stage = 0;
+        phase ^= 1u;
       }
     }
     // after a give-up, let every tile this warp requested land (bounded)

@@ -243,7 +243,7 @@ __device__ __forceinline__ void group_barrier(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-constexpr int kStages = 4;        // ring depth per warp
+constexpr int kStages = 3;        // ring depth per warp
 constexpr int kSlots = 8;         // 512-byte code chunks per stage per warp
 constexpr int kChunk = 512;       // one warp-wide 16-byte-per-lane row slice
 constexpr int kStageBytes = kSlots * (kChunk + 32);
@@ -411,7 +411,7 @@ __device__ void run_segment(const FfnArgs& a, const VExpert& ve, int r0, int r1,
 }
 
 template <int PHASE, int BPL, int RCMAX>
-__global__ void __launch_bounds__(kThreads) k_ffn_gemv(FfnArgs a, int KS, int fast_scales) {
+__global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a, int KS, int fast_scales) {
   extern __shared__ __align__(128) unsigned char smem[];
   pdl_wait();
   pdl_trigger();
@@ -447,12 +447,8 @@ __global__ void __launch_bounds__(kThreads) k_ffn_gemv(FfnArgs a, int KS, int fa
     const VExpert ve = vexpert(a, PHASE, v, nA);
     for (int t0 = 0; t0 < ve.R; t0 += RCMAX) {
       const int nt = min(RCMAX, ve.R - t0);
-      if (RCMAX >= 8 && nt > 4) {
-        run_segment<PHASE, BPL, (RCMAX >= 8 ? 8 : RCMAX)>(a, ve, r0, r1, t0, nt, wk);
-      } else if (RCMAX >= 4 && nt > 2) {
-        run_segment<PHASE, BPL, (RCMAX >= 4 ? 4 : RCMAX)>(a, ve, r0, r1, t0, nt, wk);
-      } else if (RCMAX >= 2 && nt == 2) {
-        run_segment<PHASE, BPL, (RCMAX >= 2 ? 2 : RCMAX)>(a, ve, r0, r1, t0, nt, wk);
+      if (RCMAX >= 2 && nt == 2) {
+        run_segment<PHASE, BPL, (RCMAX >= 2 ? 2 : 1)>(a, ve, r0, r1, t0, nt, wk);
       } else {
         run_segment<PHASE, BPL, 1>(a, ve, r0, r1, t0, nt, wk);
       }
@@ -472,13 +468,12 @@ inline void split_of(int K, int& KS, int& BPL) {
 }
 
 // Largest token tile per pass: x registers hold BPL * RC blocks per lane.
+// Token rows per pass: two at most (their registers stay small enough for
+// four CTAs per SM); a bucket of more tokens takes several passes over the
+// same weights, the later ones served from L2.
 inline int rcmax_of(int PHASE, int T, int BPL) {
-  int cap = PHASE == 0 ? 8 : 4;
-  cap = cap / BPL > 0 ? cap / BPL : 1;
-  const int want = T >= 8 ? 8 : T;
-  int r = 1;
-  while (r < want) r <<= 1;
-  return r < cap ? r : cap;
+  (void)PHASE;
+  return (T >= 2 && BPL <= 2) ? 2 : 1;
 }
 
 template <int PHASE, int BPL, int RCMAX>
@@ -501,15 +496,9 @@ cudaError_t launch_phase(const FfnArgs& a, int grid, cudaStream_t st) {
   if (BPL == B && RCMAX == R) return launch_one<PHASE, B, R>(a, grid, KS, fast, st);
   MOE_GEMV_CASE(1, 1)
   MOE_GEMV_CASE(1, 2)
-  MOE_GEMV_CASE(1, 4)
   MOE_GEMV_CASE(2, 1)
   MOE_GEMV_CASE(2, 2)
   MOE_GEMV_CASE(4, 1)
-  if constexpr (PHASE == 0) {
-    MOE_GEMV_CASE(1, 8)
-    MOE_GEMV_CASE(2, 4)
-    MOE_GEMV_CASE(4, 2)
-  }
 #undef MOE_GEMV_CASE
   return cudaErrorInvalidValue;
 }
@@ -552,9 +541,9 @@ int gemv_grid() {
   static int occ = 0;
   if (occ == 0) {
     int o = 0;
-    cudaFuncSetAttribute(k_ffn_gemv<0, 1, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(k_ffn_gemv<0, 1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kGemvSmem);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_ffn_gemv<0, 1, 8>, kThreads, kGemvSmem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_ffn_gemv<0, 1, 2>, kThreads, kGemvSmem);
     occ = o > 0 ? o : 1;
   }
   return device_info().sm_count * occ;
