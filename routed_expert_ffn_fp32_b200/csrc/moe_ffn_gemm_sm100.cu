@@ -13,7 +13,9 @@
 // shared expert) and per 128-row tile of its weights, one work item computes
 //   D[m, n] = sum_k W[m, k] * A[n, k]      m: weight rows, n: bucket tokens
 // with W on the MMA's M side (128 rows) and the bucket's tokens on its N side
-// (up to kBN per item), so small buckets waste no tensor work on padding.
+// (up to BN per item), so small buckets waste no tensor work on padding.
+// Two TMEM accumulator buffers let the epilogue of one item overlap the MMAs
+// of the next.
 // Phase 0: W = gate and up (two accumulators), epilogue h = silu(g) * u,
 // re-quantised to MXFP4 along I.  Phase 1: W = down, epilogue writes the
 // float32 expert outputs into `partial` rows (pair index order).
@@ -38,7 +40,6 @@ namespace moe {
 namespace {
 
 constexpr int kBM = 128;            // weight rows per item (MMA M)
-constexpr int kBN = 128;            // bucket tokens per item (max MMA N)
 constexpr int kBKB = 128;           // K bytes per stage (256 FP4 values)
 constexpr int kGemmThreads = 192;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
@@ -46,23 +47,29 @@ constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
 template <int PHASE>
 struct GemmCfg {
   static constexpr int NPROJ = PHASE == 0 ? 2 : 1;
-  static constexpr int NMB = (kBN + 127) / 128;  // 128-row blocks of B scale factors
+  // bucket tokens per item (MMA N); two accumulator buffers of NPROJ x BN
+  // columns plus the scale factors fit the 512 TMEM columns
+  static constexpr int BN = PHASE == 0 ? 112 : 128;
+  static constexpr int NMB = (BN + 127) / 128;   // 128-row blocks of B scale factors
   static constexpr int A_BYTES = kBM * kBKB;     // 16 KB per projection
-  static constexpr int B_BYTES = kBN * kBKB;
+  static constexpr int B_BYTES = BN * kBKB;
   static constexpr int SFA_BYTES = 2 * 512;      // two K atoms (8 scales) per stage
   static constexpr int SFB_BYTES = 2 * NMB * 512;
   static constexpr int STAGE_RAW = NPROJ * A_BYTES + B_BYTES + NPROJ * SFA_BYTES + SFB_BYTES;
   static constexpr int STAGE = (STAGE_RAW + 1023) / 1024 * 1024;
-  static constexpr int NS = (200 * 1024) / STAGE > 8 ? 8 : (200 * 1024) / STAGE;
-  static constexpr int SMEM = NS * STAGE + 1024 /*barriers*/ + 1024 /*alignment slack*/;
-  // TMEM columns: accumulators, then scale factors
-  static constexpr int ACC_COLS = NPROJ * kBN;
-  static constexpr int SFA_COL = ACC_COLS;                 // NPROJ * 8 columns
-  static constexpr int SFB_COL = ACC_COLS + NPROJ * 8;     // 2 * NMB * 4 columns
+  static constexpr int EPI_BYTES = PHASE == 0 ? 4 * 32 * 33 * 4 : 0;  // transpose tiles
+  static constexpr int BUDGET = 216 * 1024 - EPI_BYTES;
+  static constexpr int NS = BUDGET / STAGE > 8 ? 8 : BUDGET / STAGE;
+  static constexpr int SMEM = NS * STAGE + EPI_BYTES + 1024 /*barriers*/ + 1024 /*alignment*/;
+  // TMEM columns: two accumulator buffers, then scale factors
+  static constexpr int ACC_COLS = NPROJ * BN;
+  static constexpr int SFA_COL = 2 * ACC_COLS;              // NPROJ * 8 columns
+  static constexpr int SFB_COL = SFA_COL + NPROJ * 8;       // 2 * NMB * 4 columns
   static constexpr int USED_COLS = SFB_COL + 2 * NMB * 4;
   static constexpr int TMEM_COLS = USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64
                                  : USED_COLS <= 128 ? 128 : USED_COLS <= 256 ? 256 : 512;
   static_assert(USED_COLS <= 512, "TMEM budget");
+  static_assert(NS >= 2, "pipeline depth");
 };
 
 struct GemmArgs {
@@ -215,6 +222,7 @@ struct Item {
   int nvalid;   // tokens of this item
 };
 
+template <int BN>
 __device__ __forceinline__ Item item_of(const GemmArgs& a, int it, int nA, int nV, int MT) {
   // virtual expert: last v with item_off[v] <= it
   int lo = 0, hi = nV - 1;
@@ -238,7 +246,7 @@ __device__ __forceinline__ Item item_of(const GemmArgs& a, int it, int nA, int n
     r.row0 = a.T * a.k;
     r.R = a.T;
   }
-  r.nvalid = min(kBN, r.R - r.nt * kBN);
+  r.nvalid = min(BN, r.R - r.nt * BN);
   return r;
 }
 
@@ -253,12 +261,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* ctl = smem + C::NS * C::STAGE;
+  float* epi = reinterpret_cast<float*>(smem + C::NS * C::STAGE);  // phase 0 transpose tiles
+  unsigned char* ctl = smem + C::NS * C::STAGE + C::EPI_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(ctl);
   uint64_t* empty = full + C::NS;
-  uint64_t* acc_full = empty + C::NS;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* drain = acc_empty + 1;
+  uint64_t* acc_full = empty + C::NS;   // [2]
+  uint64_t* acc_empty = acc_full + 2;   // [2]
+  uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -268,8 +277,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(saddr(&full[s]), 2);
       mbar_init(saddr(&empty[s]), 1);
     }
-    mbar_init(saddr(acc_full), 1);
-    mbar_init(saddr(acc_empty), 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(saddr(&acc_full[b]), 1);
+      mbar_init(saddr(&acc_empty[b]), 4);
+    }
     mbar_init(saddr(drain), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -320,9 +331,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     auto prepare = [&](int g) {
       ks_n = g % nks;
       if (ks_n == 0) {
-        wn = item_of(a, int(blockIdx.x) + (g / nks) * int(gridDim.x), nA, nV, MT);
+        wn = item_of<C::BN>(a, int(blockIdx.x) + (g / nks) * int(gridDim.x), nA, nV, MT);
         arow_n = (wn.e >= 0 ? wn.e * ROWS : 0) + wn.mt * kBM;
-        brow_n = wn.row0 + wn.nt * kBN;
+        brow_n = wn.row0 + wn.nt * C::BN;
       }
       const int sc0 = ks_n * 8;  // first scale byte of the stage
 #pragma unroll
@@ -424,15 +435,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      uint32_t phase = 0;
       bool ok = true;
       const uint32_t tsfa = tmem + C::SFA_COL;
       const uint32_t tsfb = tmem + C::SFB_COL;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        const Item w = item_of(a, it, nA, nV, MT);
+      int local = 0;  // items of this CTA so far: buffer local & 1, use local >> 1
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++local) {
+        const Item w = item_of<C::BN>(a, it, nA, nV, MT);
         const int n_mma = ((w.nvalid + 7) / 8) * 8;
-        if (!mbar_wait(saddr(acc_empty), acc_phase ^ 1u, abort_flag, a.err, 200)) break;
+        const int buf = local & 1;
+        const uint32_t acc_parity = (uint32_t(local >> 1) & 1u) ^ 1u;
+        if (!mbar_wait(saddr(&acc_empty[buf]), acc_parity, abort_flag, a.err, 200)) break;
         tc_fence_after();
+        const uint32_t tacc = tmem + buf * C::ACC_COLS;
         for (int ks = 0; ks < nks; ++ks) {
           if (!mbar_wait(saddr(&full[stage]), phase, abort_flag, a.err, 201)) {
             ok = false;
@@ -460,7 +475,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int p = 0; p < NPROJ; ++p) {
               const uint64_t adesc = desc_sw128(saddr(st + p * C::A_BYTES) + kb * 32);
-              tc_mma_mxf4(tmem + p * kBN, adesc, bdesc, id, (ks | kb) != 0,
+              tc_mma_mxf4(tacc + p * C::BN, adesc, bdesc, id, (ks | kb) != 0,
                           tsfa + p * 8 + (kb >> 1) * 4, tsfb + (kb >> 1) * C::NMB * 4);
             }
           }
@@ -471,8 +486,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
         if (!ok) break;
-        tc_commit(saddr(acc_full));
-        acc_phase ^= 1u;
+        tc_commit(saddr(&acc_full[buf]));
       }
       if (!ok || *abort_flag) {
         // give-up path: let issued MMAs finish before TMEM is released
@@ -486,38 +500,56 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
-    uint32_t acc_phase = 0;
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
-      const Item w = item_of(a, it, nA, nV, MT);
-      if (!warp_wait(saddr(acc_full), acc_phase, abort_flag, a.err, 300)) break;
+    float* tile = epi + q * 32 * 33;  // 32 x 32 transpose tile (phase 0)
+    int local = 0;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++local) {
+      const Item w = item_of<C::BN>(a, it, nA, nV, MT);
+      const int buf = local & 1;
+      if (!warp_wait(saddr(&acc_full[buf]), uint32_t(local >> 1) & 1u, abort_flag, a.err, 300))
+        break;
       tc_fence_after();
+      const uint32_t tacc = tmem + buf * C::ACC_COLS;
       const int wrow = w.mt * kBM + 32 * q + lane;  // weight row of this lane
       for (int c0 = 0; c0 < w.nvalid; c0 += 32) {
-        const uint32_t taddr = tmem + (uint32_t(32 * q) << 16) + c0;
+        const uint32_t taddr = tacc + (uint32_t(32 * q) << 16) + c0;
         if constexpr (PHASE == 0) {
+          // h for 32 tokens of this lane's row, transposed through shared
+          // memory so each thread holds one token's 32 consecutive h values:
+          // exactly one MXFP4 block along I, quantised in registers
           float g[32], u[32];
           tmem_ld32(taddr, g);
-          tmem_ld32(taddr + kBN, u);
+          tmem_ld32(taddr + C::BN, u);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int n = c0 + j;
-            const float h = g[j] / (1.f + expf(-g[j])) * u[j];
-            float amax = fabsf(h);
+          for (int j = 0; j < 32; ++j) tile[lane * 33 + j] = g[j] / (1.f + expf(-g[j])) * u[j];
+          __syncwarp();
+          const int n = c0 + lane;  // token of this thread
+          if (n < w.nvalid) {
+            float hv[32];
+            float amax = 0.f;
 #pragma unroll
-            for (int off = 16; off >= 1; off >>= 1)
-              amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
-            const int X = mx_scale_exponent(amax);
-            const float hn = __shfl_down_sync(kFull, h, 1);
-            if (n < w.nvalid) {
-              const size_t orow = size_t(w.row0 + w.nt * kBN + n);
-              if ((lane & 1) == 0) {
-                const float inv = exp2i(-X);
-                a.hq[orow * (a.I / 2) + (w.mt * kBM + 32 * q) / 2 + lane / 2] =
-                    uint8_t(f32x2_to_e2m1x2(h * inv, hn * inv));
-              }
-              if (lane == 0) a.hs[orow * (a.I / 32) + (w.mt * kBM + 32 * q) / 32] = uint8_t(X + 127);
+            for (int i = 0; i < 32; ++i) {
+              hv[i] = tile[i * 33 + lane];
+              amax = fmaxf(amax, fabsf(hv[i]));
             }
+            const int X = mx_scale_exponent(amax);
+            const float inv = exp2i(-X);
+            uint32_t word[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint32_t acc = 0;
+#pragma unroll
+              for (int b = 0; b < 4; ++b)
+                acc |= f32x2_to_e2m1x2(hv[8 * j + 2 * b] * inv, hv[8 * j + 2 * b + 1] * inv)
+                       << (8 * b);
+              word[j] = acc;
+            }
+            const size_t orow = size_t(w.row0 + w.nt * C::BN + n);
+            const int i0 = w.mt * kBM + 32 * q;  // first intermediate index of the block
+            *reinterpret_cast<uint4*>(a.hq + orow * (a.I / 2) + i0 / 2) =
+                make_uint4(word[0], word[1], word[2], word[3]);
+            a.hs[orow * (a.I / 32) + i0 / 32] = uint8_t(X + 127);
           }
+          __syncwarp();
         } else {
           float o[32];
           tmem_ld32(taddr, o);
@@ -525,7 +557,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int j = 0; j < 32; ++j) {
             const int n = c0 + j;
             if (n < w.nvalid) {
-              const int r = w.nt * kBN + n;
+              const int r = w.nt * C::BN + n;
               const int prow = w.e >= 0 ? a.entries[w.row0 + r] : a.T * a.k + r;
               a.partial[size_t(prow) * a.H + wrow] = o[j];
             }
@@ -534,8 +566,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(saddr(acc_empty));
-      acc_phase ^= 1u;
+      if (lane == 0) mbar_arrive(saddr(&acc_empty[buf]));
     }
   }
 
@@ -597,51 +628,53 @@ __global__ void __launch_bounds__(256) k_act_gather(const uint16_t* x, const int
 }
 
 // ------------------------------------------------------- item prefix sums ---
-// item_off[p][v] = sum_{v' < v} MT_p * ceil(R_v' / kBN) for both phases.
+// item_off[p][v] = sum_{v' < v} MT_p * ceil(R_v' / BN_p) for both phases.
 __global__ void __launch_bounds__(1024) k_gemm_plan(const int32_t* offsets, const int32_t* plan,
                                                     int T, int k, int has_shared, int MT0, int MT1,
                                                     int32_t* item_off0, int32_t* item_off1) {
   pdl_wait();
   pdl_trigger();
-  __shared__ int tiles[kMaxExperts + 2];
-  __shared__ int wsum[33];
+  constexpr int BN0 = GemmCfg<0>::BN, BN1 = GemmCfg<1>::BN;
+  __shared__ int rows_of[kMaxExperts + 2];
   const int nA = plan[0];
   const int nV = nA + (has_shared ? 1 : 0);
   for (int v = threadIdx.x; v < nV; v += blockDim.x) {
-    int R;
     if (v < nA) {
       const int e = plan[1 + v];
-      R = offsets[e + 1] - offsets[e];
+      rows_of[v] = offsets[e + 1] - offsets[e];
     } else {
-      R = T;
+      rows_of[v] = T;
     }
-    tiles[v] = (R + kBN - 1) / kBN;
   }
   __syncthreads();
   if (threadIdx.x < 32) {
-    // one warp: running prefix in chunks of 32
-    int run = 0;
+    // one warp: running prefix sums in chunks of 32
+    int run0 = 0, run1 = 0;
     for (int base = 0; base < nV; base += 32) {
       const int v = base + threadIdx.x;
-      const int t = v < nV ? tiles[v] : 0;
-      int incl = t;
+      const int R = v < nV ? rows_of[v] : 0;
+      const int t0 = (R + BN0 - 1) / BN0 * MT0, t1 = (R + BN1 - 1) / BN1 * MT1;
+      int i0 = t0, i1 = t1;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(kFull, incl, off);
-        if ((int)threadIdx.x >= off) incl += y;
+        const int y0 = __shfl_up_sync(kFull, i0, off), y1 = __shfl_up_sync(kFull, i1, off);
+        if ((int)threadIdx.x >= off) {
+          i0 += y0;
+          i1 += y1;
+        }
       }
       if (v < nV) {
-        item_off0[v] = (run + incl - t) * MT0;
-        item_off1[v] = (run + incl - t) * MT1;
+        item_off0[v] = run0 + i0 - t0;
+        item_off1[v] = run1 + i1 - t1;
       }
-      run += __shfl_sync(kFull, incl, 31);
+      run0 += __shfl_sync(kFull, i0, 31);
+      run1 += __shfl_sync(kFull, i1, 31);
     }
     if (threadIdx.x == 0) {
-      item_off0[nV] = run * MT0;
-      item_off1[nV] = run * MT1;
+      item_off0[nV] = run0;
+      item_off1[nV] = run1;
     }
   }
-  (void)wsum;
 }
 
 // --------------------------------------------------------------- host side ---
@@ -703,9 +736,9 @@ cudaError_t launch_ffn_gemm(const FfnArgs& a, const GemmBuffers& gb, cudaStream_
   const uint64_t HB = a.H / 2, IB = a.I / 2;
   bool ok = make_map(&g0, a.ex.gq, HB, uint64_t(a.E) * a.I, kBM) &&
             make_map(&g1, a.ex.uq, HB, uint64_t(a.E) * a.I, kBM) &&
-            make_map(&bx, gb.xq, HB, rows, kBN) &&
+            make_map(&bx, gb.xq, HB, rows, GemmCfg<0>::BN) &&
             make_map(&d0, a.ex.dq, IB, uint64_t(a.E) * a.H, kBM) &&
-            make_map(&bh, gb.hq, IB, rows, kBN);
+            make_map(&bh, gb.hq, IB, rows, GemmCfg<1>::BN);
   if (a.has_shared) {
     ok = ok && make_map(&sg0, a.sh.gq, HB, a.I, kBM) && make_map(&sg1, a.sh.uq, HB, a.I, kBM) &&
          make_map(&sd0, a.sh.dq, IB, a.H, kBM);
