@@ -103,6 +103,19 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<unsigned char*>(ws) + off);
 }
 
+// CUDA-core FFN: the lane-per-row GEMV where the shape fits it, else the
+// K-split GEMV.
+cudaError_t launch_gemv_path(const FfnArgs& a, void* ws, const WsLayout& L, cudaStream_t s) {
+  const moe_shape_t shape{a.T, a.H, a.I, a.E, a.k};
+  if (a.xh != nullptr && lane_supported(shape)) {
+    const cudaError_t e = launch_ffn_lane(a, at<float>(ws, L.lane_part),
+                                          at<uint32_t>(ws, L.lane_cnt), at<int>(ws, L.lane_tab), s);
+    if (e != cudaErrorNotSupported) return e;
+  }
+  return launch_ffn_gemv(a, s);
+}
+
+
 constexpr int kFusedRouteMaxT = 32;
 
 GemmBuffers gemm_buffers(void* ws, const WsLayout& L, int E) {
@@ -231,7 +244,10 @@ moe_status_t moe_expert_ffn_mxfp4(const moe_mxfp4_experts_t* experts,
   a.has_shared = has_shared;
   a.act_mxfp4 = precision == MOE_ACT_MXFP4;
   if (rp == MOE_PATH_GEMM) return cuda_status(launch_ffn_gemm(a, gemm_buffers(ws, L, shape.E), s));
-  return cuda_status(launch_ffn_gemv(a, s));
+  a.xh = at<uint16_t>(ws, L.xh);
+  e = launch_x_f16(x, shape.T, shape.H, a.act_mxfp4, at<uint16_t>(ws, L.xh), s);
+  if (e != cudaSuccess) return cuda_status(e);
+  return cuda_status(launch_gemv_path(a, ws, L, s));
 }
 
 moe_status_t moe_combine(const float* partial, const float* topk_w, moe_shape_t shape,
@@ -283,6 +299,10 @@ moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router, const f
   r.H = shape.H;
   r.E = shape.E;
   r.k = shape.k;
+  if (rp == MOE_PATH_GEMV) {
+    r.xh = at<uint16_t>(ws, L.xh);
+    r.act_mxfp4 = precision == MOE_ACT_MXFP4;
+  }
   cudaError_t e;
   if (shape.T <= kFusedRouteMaxT) {
     e = launch_route_logits(r, true, s);
@@ -290,6 +310,7 @@ moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router, const f
     e = launch_route_logits(r, false, s);
     if (e == cudaSuccess) e = launch_topk(r, s);
     if (e == cudaSuccess) e = launch_bucket(r, s);
+    if (e == cudaSuccess && r.xh != nullptr) e = launch_x_f16(x, shape.T, shape.H, r.act_mxfp4, r.xh, s);
   }
   if (e != cudaSuccess) return cuda_status(e);
 
@@ -311,8 +332,9 @@ moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router, const f
   a.k = shape.k;
   a.has_shared = has_shared;
   a.act_mxfp4 = precision == MOE_ACT_MXFP4;
+  a.xh = r.xh;
   e = rp == MOE_PATH_GEMM ? launch_ffn_gemm(a, gemm_buffers(ws, L, shape.E), s)
-                          : launch_ffn_gemv(a, s);
+                          : launch_gemv_path(a, ws, L, s);
   if (e == cudaSuccess)
     e = launch_combine(a.partial, r.w, shape.T, shape.H, shape.k, has_shared, y, s);
   return cuda_status(e);

@@ -719,6 +719,11 @@ cudaError_t launch_gemm_phase(const GemmArgs& g, const CUtensorMap& a0, const CU
 
 }  // namespace
 
+bool make_tma_map_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
+                     uint32_t box_rows) {
+  return make_map(m, base, row_bytes, rows, box_rows);
+}
+
 bool gemm_supported(const moe_shape_t& s) {
   return s.H % 256 == 0 && s.I % 128 == 0 && encode_fn() != nullptr;
 }

@@ -170,52 +170,6 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[NVAL], int lane) {
   return v[0];
 }
 
-struct VExpert {
-  const uint8_t* q[2];
-  const uint8_t* s[2];
-  const int32_t* rows;  // pair indices of the bucket, or nullptr for the shared expert
-  int R;                // tokens
-};
-
-__device__ __forceinline__ VExpert vexpert(const FfnArgs& a, int phase, int v, int nA) {
-  VExpert ve;
-  const int K = phase == 0 ? a.H : a.I;
-  const int ROWS = phase == 0 ? a.I : a.H;
-  const size_t mat = size_t(ROWS) * (K / 2), smat = size_t(ROWS) * (K / 32);
-  if (v < nA) {
-    const int e = a.plan[1 + v];
-    const int beg = a.offsets[e], end = a.offsets[e + 1];
-    ve.rows = a.entries + beg;
-    ve.R = end - beg;
-    if (phase == 0) {
-      ve.q[0] = a.ex.gq + e * mat; ve.s[0] = a.ex.gs + e * smat;
-      ve.q[1] = a.ex.uq + e * mat; ve.s[1] = a.ex.us + e * smat;
-    } else {
-      ve.q[0] = a.ex.dq + e * mat; ve.s[0] = a.ex.ds + e * smat;
-      ve.q[1] = nullptr; ve.s[1] = nullptr;
-    }
-  } else {
-    ve.rows = nullptr;
-    ve.R = a.T;
-    if (phase == 0) {
-      ve.q[0] = a.sh.gq; ve.s[0] = a.sh.gs;
-      ve.q[1] = a.sh.uq; ve.s[1] = a.sh.us;
-    } else {
-      ve.q[0] = a.sh.dq; ve.s[0] = a.sh.ds;
-      ve.q[1] = nullptr; ve.s[1] = nullptr;
-    }
-  }
-  return ve;
-}
-
-// Output row (pair index, or T*k + t for the shared expert) of bucket row r.
-__device__ __forceinline__ int out_row(const FfnArgs& a, const VExpert& ve, int r) {
-  return ve.rows ? ve.rows[r] : a.T * a.k + r;
-}
-__device__ __forceinline__ int token_of(const FfnArgs& a, const VExpert& ve, int r) {
-  return ve.rows ? ve.rows[r] / a.k : r;
-}
-
 // ---------------------------------------------------------------------------
 // Asynchronous global -> shared copies (cp.async): each lane streams its own
 // 16-byte code chunks into a per-warp ring of stages, so several stages of
@@ -226,6 +180,10 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 }
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src)
                : "memory");
 }
 __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
@@ -535,7 +493,23 @@ __global__ void __launch_bounds__(256) k_combine(const float* partial, const flo
   *reinterpret_cast<uint2*>(y + size_t(t) * H + c) = out;
 }
 
+// bf16 token rows -> f16 (for callers that did not route through the router)
+__global__ void __launch_bounds__(256) k_x_f16(const uint16_t* x, int nblk, int act_mxfp4,
+                                               uint16_t* xh) {
+  pdl_wait();
+  pdl_trigger();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nblk; i += gridDim.x * blockDim.x)
+    bf16_block_to_f16(x + size_t(i) * 32, xh + size_t(i) * 32, act_mxfp4 != 0);
+}
+
 }  // namespace
+
+cudaError_t launch_x_f16(const uint16_t* x, int T, int H, int act_mxfp4, uint16_t* xh,
+                         cudaStream_t st) {
+  const int nblk = T * (H / 32);
+  const int grid = min(1024, (nblk + 255) / 256);
+  return launch_pdl(k_x_f16, dim3(grid), dim3(256), 0, st, x, nblk, act_mxfp4, xh);
+}
 
 int gemv_grid() {
   static int occ = 0;
@@ -550,10 +524,9 @@ int gemv_grid() {
 }
 
 cudaError_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t st) {
-  const int grid = gemv_grid();
-  cudaError_t e = launch_phase<0>(a, grid, st);
+  const cudaError_t e = launch_phase<0>(a, gemv_grid(), st);
   if (e != cudaSuccess) return e;
-  return launch_phase<1>(a, grid, st);
+  return launch_phase<1>(a, gemv_grid(), st);
 }
 
 cudaError_t launch_combine(const float* partial, const float* w, int T, int H, int k,

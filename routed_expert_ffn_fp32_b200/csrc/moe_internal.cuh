@@ -16,6 +16,12 @@ namespace moe {
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 16;
 constexpr unsigned kFull = 0xffffffffu;
+// Lane-per-row GEMV: largest batch it takes (larger ones use the K-split
+// GEMV), CTAs (one per SM, at most), warps per CTA, tokens per pass.
+constexpr int kLaneMaxT = 64;
+constexpr int kLaneMaxCtas = 160;
+constexpr int kLaneWarps = 8;
+constexpr int kLaneRMax = 8;
 
 // ---------------------------------------------------------------------------
 // Workspace layout.  Every region starts on a 256-byte boundary.
@@ -30,8 +36,13 @@ struct WsLayout {
   size_t offsets;   // i32 [E + 1]
   size_t entries;   // i32 [T * k]
   size_t plan;      // i32 [E + 2]: [0] active experts, [1..] their ids (ascending)
+  size_t xh;        // f16 [T, H]  token rows as f16 (MXFP4-rounded in that mode)
   size_t h;         // f32 [T*k + S*T, I]   SwiGLU output rows (by pair index)
   size_t partial;   // f32 [T*k + S*T, H]   expert output rows (by pair index)
+  // lane-per-row GEMV (T <= kLaneMaxT)
+  size_t lane_part;  // f32 [warps][2][kLaneRMax][2][32]  split row-block partial sums
+  size_t lane_cnt;   // u32 [row blocks]  split row-block arrivals  } zero between calls;
+  size_t lane_tab;   // i32 [row blocks][atoms]  contributors   } each call leaves them zero
   // tensor-core path only
   size_t xq, xs;    // u8 [rows, H/2], [rows, H/32]  MXFP4 token rows, bucket order
   size_t hq, hs;    // u8 [rows, I/2], [rows, I/32]  MXFP4 SwiGLU rows, bucket order
@@ -57,8 +68,16 @@ inline WsLayout ws_layout(const moe_shape_t& s, int has_shared, int gemm) {
   L.offsets = take((E + 1) * 4);
   L.entries = take(T * k * 4);
   L.plan = take((E + 2) * 4);
+  L.xh = take(T * H * 2);
   L.h = take(rows * I * 4);
   L.partial = take(rows * H * 4);
+  const bool lane = T <= size_t(kLaneMaxT);
+  L.lane_part = take(lane ? size_t(kLaneMaxCtas) * kLaneWarps * 2 * kLaneRMax * 2 * 32 * 4 : 0);
+  // passes: at most one per virtual expert plus one per kLaneRMax rows
+  const size_t passes = E + 1 + (rows + kLaneRMax - 1) / kLaneRMax;
+  const size_t rb0 = I / 32, na0 = (H + 255) / 256, rb1 = H / 32, na1 = (I + 255) / 256;
+  L.lane_cnt = take(lane ? passes * (rb0 > rb1 ? rb0 : rb1) * 4 : 0);
+  L.lane_tab = take(lane ? passes * (rb0 * na0 > rb1 * na1 ? rb0 * na0 : rb1 * na1) * 4 : 0);
   if (gemm) {
     L.xq = take(rows * H / 2);
     L.xs = take(rows * H / 32);
@@ -168,14 +187,60 @@ __device__ __forceinline__ void pdl_trigger() {
 __device__ __forceinline__ int mx_scale_exponent(float amax) {
   const uint32_t bits = __float_as_uint(amax) & 0x7fffffffu;
   const int ef = int(bits >> 23);  // biased exponent; 0 for zero and subnormals
-  if (ef == 0) return -127;        // floor(log2 amax) - 2 < -127: clamps
-  const int X = ef - 127 - 2;
-  return X > 127 ? 127 : X;
+  const int X = ef - 127 - 2;     // ef = 0: zero or subnormal, below the clamp
+  return X < -127 ? -127 : (X > 127 ? 127 : X);
 }
 
 // 2^e as a float for e in [-127, 127] (e = -127 is the subnormal 2^-127).
 __device__ __forceinline__ float exp2i(int e) {
   return e >= -126 ? __uint_as_float(uint32_t(e + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// 32 bf16 values -> 32 f16 values (exact for |v| >= 2^-17 and |v| <= 65504);
+// with mx the block is first rounded through MXFP4 (OCP scale, RNE, saturate).
+__device__ __forceinline__ void bf16_block_to_f16(const uint16_t* src, uint16_t* dst, bool mx) {
+  float f[32];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 v = *reinterpret_cast<const uint4*>(src + 8 * q);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      f[8 * q + 2 * j] = bf16_bits_to_f32(w[j] & 0xffffu);
+      f[8 * q + 2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+    }
+  }
+  if (mx) {
+    float amax = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(f[j]));
+    const int X = mx_scale_exponent(amax);
+    const float inv = exp2i(-X), sc = exp2i(X);
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) {
+      uint32_t byte4 = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        byte4 |= f32x2_to_e2m1x2(f[j + 2 * b] * inv, f[j + 2 * b + 1] * inv) << (8 * b);
+      uint32_t h2[4];
+      e2m1x8_to_f16x2(byte4, h2);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const float2 d = f16x2_to_f32x2(h2[b]);
+        f[j + 2 * b] = d.x * sc;
+        f[j + 2 * b + 1] = d.y * sc;
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 o;
+    o.x = f32x2_to_f16x2(f[8 * q + 0], f[8 * q + 1]);
+    o.y = f32x2_to_f16x2(f[8 * q + 2], f[8 * q + 3]);
+    o.z = f32x2_to_f16x2(f[8 * q + 4], f[8 * q + 5]);
+    o.w = f32x2_to_f16x2(f[8 * q + 6], f[8 * q + 7]);
+    *reinterpret_cast<uint4*>(dst + 8 * q) = o;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -192,6 +257,8 @@ struct ExpertPtrs {
 
 struct RouteArgs {
   const uint16_t* x;
+  uint16_t* xh;       // optional: f16 copy of x written by the router (decode path)
+  int act_mxfp4;      // round xh through MXFP4 first
   const float* w_router;
   const float* bias;
   float* logits;
@@ -210,6 +277,7 @@ struct FfnArgs {
   ExpertPtrs ex;
   ExpertPtrs sh;  // shared expert (n = 1) when has_shared
   const uint16_t* x;
+  const uint16_t* xh;   // f16 token rows [T, H] (decode path)
   const int32_t* offsets;
   const int32_t* entries;
   const int32_t* plan;
@@ -222,6 +290,56 @@ struct FfnArgs {
   int has_shared;
   int act_mxfp4;
 };
+
+// ---------------------------------------------------------------------------
+// Virtual experts of the FFN kernels: v < plan[0] is the v-th active routed
+// expert (its bucket rows), v = plan[0] the shared expert (all T tokens).
+// ---------------------------------------------------------------------------
+struct VExpert {
+  const uint8_t* q[2];
+  const uint8_t* s[2];
+  const int32_t* rows;  // pair indices of the bucket, or nullptr for the shared expert
+  int R;                // tokens
+};
+
+__device__ __forceinline__ VExpert vexpert(const FfnArgs& a, int phase, int v, int nA) {
+  VExpert ve;
+  const int K = phase == 0 ? a.H : a.I;
+  const int ROWS = phase == 0 ? a.I : a.H;
+  const size_t mat = size_t(ROWS) * (K / 2), smat = size_t(ROWS) * (K / 32);
+  if (v < nA) {
+    const int e = a.plan[1 + v];
+    const int beg = a.offsets[e], end = a.offsets[e + 1];
+    ve.rows = a.entries + beg;
+    ve.R = end - beg;
+    if (phase == 0) {
+      ve.q[0] = a.ex.gq + e * mat; ve.s[0] = a.ex.gs + e * smat;
+      ve.q[1] = a.ex.uq + e * mat; ve.s[1] = a.ex.us + e * smat;
+    } else {
+      ve.q[0] = a.ex.dq + e * mat; ve.s[0] = a.ex.ds + e * smat;
+      ve.q[1] = nullptr; ve.s[1] = nullptr;
+    }
+  } else {
+    ve.rows = nullptr;
+    ve.R = a.T;
+    if (phase == 0) {
+      ve.q[0] = a.sh.gq; ve.s[0] = a.sh.gs;
+      ve.q[1] = a.sh.uq; ve.s[1] = a.sh.us;
+    } else {
+      ve.q[0] = a.sh.dq; ve.s[0] = a.sh.ds;
+      ve.q[1] = nullptr; ve.s[1] = nullptr;
+    }
+  }
+  return ve;
+}
+
+// Output row (pair index, or T*k + t for the shared expert) of bucket row r.
+__device__ __forceinline__ int out_row(const FfnArgs& a, const VExpert& ve, int r) {
+  return ve.rows ? ve.rows[r] : a.T * a.k + r;
+}
+__device__ __forceinline__ int token_of(const FfnArgs& a, const VExpert& ve, int r) {
+  return ve.rows ? ve.rows[r] / a.k : r;
+}
 
 // ---------------------------------------------------------------------------
 // Launchers (return cudaError_t of the launch)
@@ -239,6 +357,13 @@ cudaError_t launch_bucket(const RouteArgs& a, cudaStream_t st);
 cudaError_t launch_plan(const RouteArgs& a, cudaStream_t st);
 
 cudaError_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t st);
+// Lane-per-row GEMV of both phases; cudaErrorNotSupported when the shape does
+// not fit it (the caller then uses launch_ffn_gemv).
+cudaError_t launch_ffn_lane(const FfnArgs& a, float* lane_part, uint32_t* lane_cnt,
+                            int* lane_tab, cudaStream_t st);
+bool lane_supported(const moe_shape_t& s);
+cudaError_t launch_x_f16(const uint16_t* x, int T, int H, int act_mxfp4, uint16_t* xh,
+                         cudaStream_t st);
 
 struct GemmBuffers {
   uint8_t* xq;

@@ -18,8 +18,10 @@
 //     H/128 + 9 roundings (lane chain, 5 shuffle levels, 3 quarter sums, the
 //     bias), the bound the parity tests use for near-ties.
 //     With fuse_tail the CTA that finishes last (arrival counter in the
-//     workspace, reset to zero by that CTA) runs top-k and the bucket for the
-//     whole batch, so a decode step routes in one launch.
+//     workspace, reset to zero by that CTA) runs top-k (a warp per token) and
+//     a one-warp bucket for the whole batch, so a decode step routes in one
+//     launch.
+//   k_route_logits_tiled: batches of more than 32 tokens (see the kernel).
 //   k_topk: one warp per token.
 //   k_bucket: one CTA; counts by shared-memory atomics, exclusive scan, then a
 //     stable placement of each 1024-pair chunk: ranks among equal experts come
@@ -252,6 +254,64 @@ __device__ void bucket_block(const int32_t* idx, int npairs, int E, int32_t* cou
   }
 }
 
+// One-warp stable bucket for small batches (the decode tail): counts by
+// shared-memory atomics, warp scans over the experts, then pairs placed in
+// order, ranks among equal experts from __match_any_sync.  No block barrier.
+__device__ void bucket_warp(const int32_t* idx, int npairs, int E, int32_t* counts,
+                            int32_t* offsets, int32_t* entries, int32_t* plan, int* err, int* cnt,
+                            int* cur) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int e = lane; e < E; e += 32) cnt[e] = 0;
+  __syncwarp();
+  for (int p = lane; p < npairs; p += 32) {
+    const int e = idx[p];
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+    else latch_error(err, MOE_ERR_DEVICE_DATA, p);
+  }
+  __syncwarp();
+  int run = 0, run_act = 0;
+  for (int base = 0; base < E; base += 32) {
+    const int e = base + lane;
+    const int c = e < E ? cnt[e] : 0;
+    const int act = c > 0;
+    int incl = c, incl_act = act;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(kFull, incl, off), ya = __shfl_up_sync(kFull, incl_act, off);
+      if (lane >= off) {
+        incl += y;
+        incl_act += ya;
+      }
+    }
+    if (e < E) {
+      const int ex = run + incl - c;
+      counts[e] = c;
+      offsets[e] = ex;
+      cur[e] = ex;
+      if (act) plan[1 + run_act + incl_act - 1] = e;
+    }
+    run += __shfl_sync(kFull, incl, 31);
+    run_act += __shfl_sync(kFull, incl_act, 31);
+  }
+  if (lane == 0) {
+    offsets[E] = run;
+    plan[0] = run_act;
+  }
+  __syncwarp();
+  for (int base = 0; base < npairs; base += 32) {
+    const int p = base + lane;
+    const int e = p < npairs ? idx[p] : -1;
+    const bool valid = e >= 0 && e < E;
+    const unsigned grp = __match_any_sync(kFull, valid ? e : (E + lane));
+    const int rank = __popc(grp & lt_mask);
+    if (valid) entries[cur[e] + rank] = p;
+    __syncwarp();
+    if (valid && rank == 0) cur[e] += __popc(grp);
+    __syncwarp();
+  }
+}
+
 // ---------------------------------------------------------------- kernels ---
 template <int TT>
 __global__ void __launch_bounds__(kRouteThreads) k_route_logits(RouteArgs a, int fuse_tail) {
@@ -272,6 +332,15 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_logits(RouteArgs a, int
     for (int i = tid; i < nt * vec_per_row; i += kRouteThreads) dst[i] = __ldg(src + i);
   }
   __syncthreads();
+  if (a.xh != nullptr && blockIdx.x == 0) {
+    // f16 copy of the token rows for the expert GEMV (one 32-value block per thread)
+    const int nblk = nt * (H / 32);
+    for (int i = tid; i < nblk; i += kRouteThreads) {
+      const int t = i / (H / 32), b = i % (H / 32);
+      bf16_block_to_f16(xs + size_t(t) * H + 32 * b, a.xh + size_t(t0 + t) * H + 32 * b,
+                        a.act_mxfp4 != 0);
+    }
+  }
   const int e = blockIdx.x * 2 + (warp >> 2);
   const int quarter = warp & 3;
   const int qlen = H / 4;  // multiple of 8
@@ -343,9 +412,111 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_logits(RouteArgs a, int
   int32_t* idx_s = reinterpret_cast<int32_t*>(smem);  // reuse: [T*k]
   topk_block(a, idx_s);
   __syncthreads();
-  BucketSmem bs = bucket_smem(smem + align_up16(size_t(a.T) * a.k * 4), a.E, kRouteThreads / 32);
-  bucket_block(idx_s, a.T * a.k, a.E, a.counts, a.offsets, a.entries, a.plan, a.err, bs);
-  if (tid == 0) *a.counter = 0u;
+  if (warp == 0) {
+    int* cnt = reinterpret_cast<int*>(smem + align_up16(size_t(a.T) * a.k * 4));
+    bucket_warp(idx_s, a.T * a.k, a.E, a.counts, a.offsets, a.entries, a.plan, a.err, cnt,
+                cnt + a.E);
+    if (lane == 0) *a.counter = 0u;
+  }
+}
+
+// Router logits for prefill-sized batches: a 64-token x 64-expert tile per
+// CTA, K in chunks of 32 staged in shared memory (double buffered), each
+// thread a 4 x 4 register tile.  Products of a chunk are summed into a fresh
+// register and chunk sums are added to the running total, so every product
+// meets at most 32 + H/32 + 1 roundings (the bound the parity tests use).
+constexpr int kTileT = 64, kTileE = 64, kTileK = 32;
+
+__global__ void __launch_bounds__(256) k_route_logits_tiled(RouteArgs a) {
+  __shared__ __align__(16) float xs[2][kTileK][kTileT + 4];  // [k][token]
+  __shared__ __align__(16) float wsm[2][kTileK][kTileE + 4]; // [k][expert]
+  pdl_wait();
+  pdl_trigger();
+  const int tid = threadIdx.x;
+  const int t0 = blockIdx.y * kTileT, e0 = blockIdx.x * kTileE;
+  const int ty = tid / 16, tx = tid % 16;  // 4 tokens ty*4.., 4 experts tx*4..
+  const int H = a.H;
+  const int nchunks = H / kTileK;
+  // global -> register staging: each thread loads 8 bf16 of x and 8 floats of W
+  const int lr = tid / 4, lc = (tid % 4) * 8;  // row (token / expert) and first k
+  uint4 xreg;
+  float4 wreg0, wreg1;
+  auto gload = [&](int ck) {
+    const int k0 = ck * kTileK + lc;
+    const int t = t0 + lr, e = e0 + lr;
+    xreg = (t < a.T) ? __ldg(reinterpret_cast<const uint4*>(a.x + size_t(t) * H + k0))
+                     : make_uint4(0, 0, 0, 0);
+    if (e < a.E) {
+      wreg0 = __ldg(reinterpret_cast<const float4*>(a.w_router + size_t(e) * H + k0));
+      wreg1 = __ldg(reinterpret_cast<const float4*>(a.w_router + size_t(e) * H + k0 + 4));
+    } else {
+      wreg0 = wreg1 = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto sstore = [&](int buf) {
+    const uint32_t xw[4] = {xreg.x, xreg.y, xreg.z, xreg.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      xs[buf][lc + 2 * j][lr] = bf16_bits_to_f32(xw[j] & 0xffffu);
+      xs[buf][lc + 2 * j + 1][lr] = bf16_bits_to_f32(xw[j] >> 16);
+    }
+    wsm[buf][lc + 0][lr] = wreg0.x;
+    wsm[buf][lc + 1][lr] = wreg0.y;
+    wsm[buf][lc + 2][lr] = wreg0.z;
+    wsm[buf][lc + 3][lr] = wreg0.w;
+    wsm[buf][lc + 4][lr] = wreg1.x;
+    wsm[buf][lc + 5][lr] = wreg1.y;
+    wsm[buf][lc + 6][lr] = wreg1.z;
+    wsm[buf][lc + 7][lr] = wreg1.w;
+  };
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  gload(0);
+  sstore(0);
+  __syncthreads();
+  for (int ck = 0; ck < nchunks; ++ck) {
+    const int buf = ck & 1;
+    if (ck + 1 < nchunks) gload(ck + 1);
+    float part[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) part[i][j] = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < kTileK; ++k) {
+      const float4 xv = *reinterpret_cast<const float4*>(&xs[buf][k][ty * 4]);
+      const float4 wv = *reinterpret_cast<const float4*>(&wsm[buf][k][tx * 4]);
+      const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
+      const float wa[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(xa[i], wa[j], part[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
+    if (ck + 1 < nchunks) sstore(buf ^ 1);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= a.T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e < a.E) {
+        float v = acc[i][j];
+        if (a.bias) v += __ldg(a.bias + e);
+        a.logits[size_t(t) * a.E + e] = v;
+      }
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kRouteThreads) k_topk(RouteArgs a) {
@@ -390,10 +561,14 @@ __global__ void __launch_bounds__(kBucketThreads) k_plan(RouteArgs a) {
 static size_t route_smem(int TT, int H) { return size_t(TT) * H * 2 + 8 * TT * 4; }
 
 cudaError_t launch_route_logits(const RouteArgs& a, bool fuse_tail, cudaStream_t st) {
+  if (!fuse_tail && a.T > 32) {
+    dim3 grid((a.E + kTileE - 1) / kTileE, (a.T + kTileT - 1) / kTileT);
+    return launch_pdl(k_route_logits_tiled, grid, dim3(256), 0, st, a);
+  }
   const int TT = a.T <= 1 ? 1 : (a.T <= 2 ? 2 : (a.T <= 4 ? 4 : 8));
   size_t smem = route_smem(TT, a.H);
   if (fuse_tail) {
-    const size_t tail = align_up16(size_t(a.T) * a.k * 4) + bucket_smem_bytes(a.E, kRouteThreads);
+    const size_t tail = align_up16(size_t(a.T) * a.k * 4) + size_t(a.E) * 8;
     smem = smem > tail ? smem : tail;
   }
   dim3 grid((a.E + 1) / 2, (a.T + TT - 1) / TT);
@@ -415,7 +590,7 @@ cudaError_t launch_route_logits(const RouteArgs& a, bool fuse_tail, cudaStream_t
 size_t route_fused_smem(int T, int H, int E, int k) {
   const int TT = T <= 1 ? 1 : (T <= 2 ? 2 : (T <= 4 ? 4 : 8));
   const size_t a = route_smem(TT, H);
-  const size_t b = align_up16(size_t(T) * k * 4) + bucket_smem_bytes(E, kRouteThreads);
+  const size_t b = align_up16(size_t(T) * k * 4) + size_t(E) * 8;
   return a > b ? a : b;
 }
 

@@ -11,10 +11,12 @@ TOL_Y = 2e-3
 TOL_W = 1e-5
 
 
-def route_depth(H: int) -> int:
-    """Roundings any router product meets in the route kernel (lane chain of
-    H/128 products, 5 shuffle levels, 3 quarter sums, the bias)."""
-    return H // 128 + 9
+def route_depth(H: int, T: int = 1) -> int:
+    """Roundings any router product meets in the route kernels: up to 32
+    tokens, a lane chain of H/128 products, 5 shuffle levels, 3 quarter sums
+    and the bias; above 32 tokens, a 32-product chunk, H/32 chunk sums and the
+    bias."""
+    return H // 128 + 9 if T <= 32 else 32 + H // 32 + 1
 
 
 def to_dev_bits(a: np.ndarray) -> torch.Tensor:
@@ -57,11 +59,14 @@ def gpu_layer(L: dict, D: dict, cfg, path=moe.MOE_PATH_AUTO, precision=moe.MOE_A
     return {"y": bits_np(y), "idx": idx.cpu().numpy(), "w": w.cpu().numpy(), "ws": ws}
 
 
-def check_routing(L, ref, idx, w, k, H):
+def check_routing(L, ref, idx, w, k, H, T_route=None):
     """idx bit-exact except near-ties (which must still be a valid top-k);
-    w within TOL_W where idx agrees.  Returns the near-tie token indices."""
+    w within TOL_W where idx agrees.  T_route: the batch size the GPU routed
+    (selects the kernel's summation bound; default idx rows).  Returns the
+    near-tie token indices."""
     x = O.bf16_bits_to_f64(L["x"])
-    ties = O.near_tie_tokens(x, L["W_r"], L["bias"], ref["logits"], k, route_depth(H))
+    T_route = idx.shape[0] if T_route is None else T_route
+    ties = O.near_tie_tokens(x, L["W_r"], L["bias"], ref["logits"], k, route_depth(H, T_route))
     clear = np.setdiff1d(np.arange(idx.shape[0]), ties)
     np.testing.assert_array_equal(idx[clear], ref["idx"][clear])
     np.testing.assert_allclose(w[clear], ref["w"][clear], atol=TOL_W, rtol=0)

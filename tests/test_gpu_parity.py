@@ -88,7 +88,7 @@ def test_route_topk(name, T):
     iref, wref = O.route_topk(lref, cfg.k)
     # logits within the float32 error bound of the kernel's summation
     u = 2.0 ** -24
-    d = route_depth(cfg.H)
+    d = route_depth(cfg.H, T)
     bound = d * u / (1 - d * u) * (np.abs(xf) @ np.abs(W_r.astype(np.float64)).T) + 2 * u * np.abs(lref)
     if bias is not None:
         bound += u * np.abs(bias)
