@@ -7,7 +7,7 @@
 // stream of MXFP4 weights past a handful of token vectors.
 //
 // Work decomposition.  A projection's weight matrix [ROWS, K] is cut into
-// row blocks of 32 rows and, along K, into atoms of 256 values (128 code
+// row blocks of 32 rows and, along K, into atoms of 128 values (64 code
 // bytes per row).  The atoms of all (virtual expert, pass, row block) triples
 // form one flat index space, atom fastest; every warp of the grid takes a
 // contiguous range of it of equal cost, an atom of a pass with R tokens
@@ -16,13 +16,13 @@
 // with are the same for all 32 lanes (one broadcast load serves the warp).
 //
 // Data movement.  Each warp keeps D slots of shared memory.  A slot holds the
-// 32 x 128-byte code box of an atom per projection, loaded by a TMA tile copy
-// (128-byte swizzle, so the 32 lanes' 16-byte reads of one row each fall in
-// distinct banks), and the atom's 256 values of each of the pass's tokens,
-// loaded by 1-D bulk copies; all complete on the slot's mbarrier.  The copy
-// for stage j + D is issued as soon as stage j has been consumed.  The lanes
-// fetch their rows' 8 scale bytes of stage j + 1 into registers while stage j
-// computes (loads that do not allocate in L1).
+// 32 x 64-byte code box of an atom per projection, loaded by a TMA tile copy
+// (64-byte swizzle, so the 16-byte reads of any 8 consecutive rows fall in
+// distinct banks), and the atom's 128 values of each of the pass's tokens,
+// loaded by 1-D bulk copies, and each row's 4 scale bytes per projection,
+// loaded by the row's lane with cp.async; all complete on the slot's
+// mbarrier.  The copy for stage j + D is issued as soon as stage j has been
+// consumed.
 //
 // Tokens.  A pass handles up to kRMax tokens of an expert; an expert with
 // more tokens has one row block per pass in the flat index space (its weights
@@ -42,21 +42,37 @@
 // MOE_ERR_TIMEOUT, lets its in-flight copies land and returns.
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "moe_internal.cuh"
 
 namespace moe {
 
-bool make_tma_map_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
-                     uint32_t box_rows);
+bool make_tma_map_u8_box(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
+                         uint32_t box_bytes, uint32_t box_rows);
 
 namespace {
 
 constexpr int kLW = kLaneWarps;          // warps per CTA, one CTA per SM
 constexpr int kLThreads = 32 * kLW;
 constexpr int kRMax = kLaneRMax;         // tokens per pass
-constexpr int kAtomVals = 256;           // weights of a row per atom
-constexpr int kAtomCode = 128;           // code bytes of a row per atom
-constexpr int kBox = 32 * kAtomCode;     // one projection's 32-row box
+#ifndef MOE_LANE_ATOM
+#define MOE_LANE_ATOM 128
+#endif
+#ifndef MOE_LANE_SLOTS
+#define MOE_LANE_SLOTS 3
+#endif
+constexpr int kAtomVals = MOE_LANE_ATOM;  // weights of a row per atom (128 or 256)
+constexpr int kAtomCode = kAtomVals / 2;  // code bytes of a row per atom (64 or 128)
+constexpr int kBlk = kAtomVals / 32;      // scale blocks per atom
+constexpr int kBox = 32 * kAtomCode;      // one projection's 32-row box
+static_assert(kAtomVals == 128 || kAtomVals == 256, "atom width");
+
+// 16-byte chunk j of row r inside a box: the TMA swizzle (64 or 128 bytes)
+// XORs the chunk index with address bits 7..8 or 7..9.
+__device__ __forceinline__ int swz(int lane) {
+  return kAtomCode == 64 ? (lane >> 1) & 3 : lane & 7;
+}
 constexpr unsigned long long kLWaitNs = 2000000000ull;
 
 constexpr int kPfxMax = 258;             // per-expert table entries (virtual experts + 1)
@@ -65,12 +81,15 @@ constexpr int kPfxMax = 258;             // per-expert table entries (virtual ex
 // then the slots from the next 1024-byte boundary.
 template <int NPROJ>
 struct LaneCfg {
-  static constexpr int D = 2;                     // slots per warp
+  static constexpr int D = MOE_LANE_SLOTS;        // slots per warp
   static constexpr int CODE = NPROJ * kBox;       // code bytes per slot
-  static constexpr int XB = NPROJ == 2 ? 512 : 1024;  // token bytes per atom (f16 / f32)
-  static constexpr int SLOT = CODE + kRMax * XB;  // a multiple of 1024
+  static constexpr int XB = kAtomVals * (NPROJ == 2 ? 2 : 4);  // token bytes per atom
+  static constexpr int SC_OFF = CODE + kRMax * XB;  // scale bytes: [NPROJ][32 rows][kBlk]
+  static constexpr int SC = 32 * kBlk;              // scale bytes per projection
+  static constexpr int ALIGN = kAtomCode == 64 ? 512 : 1024;  // swizzle span
+  static constexpr int SLOT = (SC_OFF + 2 * SC + ALIGN - 1) / ALIGN * ALIGN;
   static constexpr int SLOTS = kLW * D;
-  static constexpr int HEAD = SLOTS * 8 + 3 * kPfxMax * 4 + 64;
+  static constexpr int HEAD = SLOTS * 8 + 3 * kPfxMax * 4 + 2 * kLW * 4;
   static constexpr int SMEM = 1024 + HEAD + SLOTS * SLOT;
 };
 static_assert(LaneCfg<2>::SMEM + 1024 <= 227 * 1024, "shared memory per block");
@@ -128,18 +147,14 @@ __device__ __forceinline__ void lane_tma(uint32_t dst, const CUtensorMap* map, i
       : "memory");
 }
 // Loads that do not allocate in L1 (scale bytes: each 32-byte sector serves
-// four atoms of one row, L2 keeps it between them).
-__device__ __forceinline__ uint2 ldg_na8(const void* p) {
-  uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
-               : "=r"(v.x), "=r"(v.y)
-               : "l"(p));
-  return v;
-}
+// eight atoms of one row, L2 keeps it between them).
 __device__ __forceinline__ uint32_t ldg_na4(const void* p) {
   uint32_t v;
   asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
   return v;
+}
+__device__ __forceinline__ void lane_cp4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void lane_bulk(uint32_t dst, const void* src, uint32_t bytes,
                                           uint32_t bar) {
@@ -157,6 +172,9 @@ __device__ __forceinline__ float2 lane_ffma2(float2 a, float2 b, float2 c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
   return make_float2(__uint_as_float(uint32_t(rd)), __uint_as_float(uint32_t(rd >> 32)));
 }
+// scale bytes of a lane's row for one atom: kBlk bytes
+using ScaleWord = std::conditional_t<kBlk == 4, uint32_t, uint2>;
+__device__ __forceinline__ uint32_t scale_byte(uint32_t s, int j) { return (s >> (8 * j)) & 0xffu; }
 __device__ __forceinline__ uint32_t scale_byte(uint2 s, int j) {
   return ((j < 4 ? s.x : s.y) >> (8 * (j & 3))) & 0xffu;
 }
@@ -271,13 +289,23 @@ struct LaneWarp {
   int nA, nV, K, ROWS, nb, lane;
   int gw, A0, A1;           // this warp's index in the grid and atom range
   LaneIt nxt;               // next stage to load
-  LaneIt look;              // stage after the one being computed
-  uint2 scn[NPROJ];         // scale bytes of stage `look` (in flight)
   int jc, ji;               // stages consumed / issued (ji counts empty tail slots)
   int jv;                   // stages issued with a copy in flight
   int ev, ee;               // expert id of virtual expert ev (cache)
-  int iv;                   // virtual expert of `ive` (cache for issue())
-  VExpert ive;
+  int iv, ipass;            // (virtual expert, pass) of the cached token rows below
+  int iR;                   // tokens of that pass
+  const void* ixsrc;        // lane t < iR: its token's value row (f16 x or f32 h)
+  // per segment being loaded: first atom, TMA row, maps, this lane's scale rows
+  int iseg, iy;
+  const CUtensorMap* imap;
+  const uint8_t* isrc[NPROJ];
+  int islot;                // ji % D
+  // prologue of the down projection: token-row copies deferred until the
+  // SwiGLU rows of the previous kernel are complete
+  const void* dsrc[C::D];
+  uint32_t ddst[C::D], dbytes[C::D], dfb[C::D];
+  int cslot;                // jc % D
+  uint32_t cpar;            // (jc / D) & 1
 
   __device__ __forceinline__ int expert(int v) {
     if (v != ev) {
@@ -287,48 +315,104 @@ struct LaneWarp {
     return ee;
   }
 
-  // Load stage ji (if any) into slot ji % D: the code boxes, and the atom's
-  // values of the pass's tokens.
-  __device__ __forceinline__ void issue() {
-    const int d = ji % C::D;
-    if (nxt.valid) {
-      const int atom = nxt.a - nxt.blk * l->NA;
-      const int e = expert(nxt.v);
-      const bool sh = e < 0;
-      const int y = (sh ? 0 : e * ROWS) + nxt.rb * 32;
-      if (nxt.v != iv) {
-        iv = nxt.v;
-        ive = vexpert(*a, PHASE, iv, nA);
+  // Per-segment state of the stage loads (nxt entered a new segment).
+  __device__ __forceinline__ void refresh() {
+    iseg = nxt.seg0;
+    const int e = expert(nxt.v);
+    const bool sh = e < 0;
+    iy = (sh ? 0 : e * ROWS) + nxt.rb * 32;
+    imap = maps + (sh ? NPROJ : 0);
+    if (nxt.v != iv || nxt.pass != ipass) {
+      iv = nxt.v;
+      ipass = nxt.pass;
+      const VExpert ve = vexpert(*a, PHASE, iv, nA);
+      const int t0 = ipass * kRMax;
+      iR = min(kRMax, ve.R - t0);
+      ixsrc = nullptr;
+      if (lane < iR) {
+        if constexpr (PHASE == 0)
+          ixsrc = a->xh + size_t(token_of(*a, ve, t0 + lane)) * a->H;
+        else
+          ixsrc = a->h + size_t(out_row(*a, ve, t0 + lane)) * a->I;
       }
-      const int t0 = nxt.pass * kRMax;
-      const int R = min(kRMax, ive.R - t0);
+    }
+    const size_t row = size_t(nxt.rb * 32 + lane);
+#pragma unroll
+    for (int pj = 0; pj < NPROJ; ++pj) {
+      const uint8_t* sbase;
+      if (PHASE == 0)
+        sbase = sh ? (pj == 0 ? a->sh.gs : a->sh.us) : (pj == 0 ? a->ex.gs : a->ex.us);
+      else
+        sbase = sh ? a->sh.ds : a->ex.ds;
+      if (!sh) sbase += size_t(e) * ROWS * nb;
+      isrc[pj] = sbase + row * nb;
+    }
+  }
+
+  // Load stage ji (if any) into slot ji % D: the code boxes, the atom's values
+  // of the pass's tokens, and the rows' scale bytes.  DJ >= 0: a prologue
+  // stage (ji == DJ) whose token-row copy is kept for flush_deferred().
+  template <int DJ = -1>
+  __device__ __forceinline__ void issue() {
+    if (nxt.valid) {
+      if (nxt.seg0 != iseg) refresh();
+      const int atom = nxt.a - nxt.blk * l->NA;
       const int kbase = atom * kAtomVals;
-      const uint32_t xbytes = uint32_t(min(kAtomVals, K - kbase)) * (PHASE == 0 ? 2 : 4);
-      const uint32_t fb = lsm(&full[d]);
-      const uint32_t dst = lsm(codes + size_t(d) * C::SLOT);
+      const bool whole = kbase + kAtomVals <= K;
+      const uint32_t xbytes =
+          (whole ? uint32_t(kAtomVals) : uint32_t(K - kbase)) * (PHASE == 0 ? 2 : 4);
+      const uint32_t fb = lsm(&full[islot]);
+      const uint32_t dst = lsm(codes + size_t(islot) * C::SLOT);
       // this slot's previous contents were read through the generic proxy
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       if (lane == 0) {
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(fb),
-                     "r"(uint32_t(NPROJ * kBox) + uint32_t(R) * xbytes)
+                     "r"(uint32_t(NPROJ * kBox) + uint32_t(iR) * xbytes)
                      : "memory");
 #pragma unroll
         for (int pj = 0; pj < NPROJ; ++pj)
-          lane_tma(dst + pj * kBox, &maps[(sh ? NPROJ : 0) + pj], atom * kAtomCode, y, fb);
+          lane_tma(dst + pj * kBox, imap + pj, atom * kAtomCode, iy, fb);
       }
       __syncwarp();
-      if (lane < R) {
-        const void* src;
-        if constexpr (PHASE == 0)
-          src = a->xh + size_t(token_of(*a, ive, t0 + lane)) * a->H + kbase;
-        else
-          src = a->h + size_t(out_row(*a, ive, t0 + lane)) * a->I + kbase;
-        lane_bulk(dst + C::CODE + lane * C::XB, src, xbytes, fb);
+      const void* xsrc =
+          lane < iR
+              ? static_cast<const unsigned char*>(ixsrc) + size_t(kbase) * (PHASE == 0 ? 2 : 4)
+              : nullptr;
+      if constexpr (DJ >= 0) {
+        dsrc[DJ] = xsrc;
+        ddst[DJ] = dst + C::CODE + lane * C::XB;
+        dbytes[DJ] = xbytes;
+        dfb[DJ] = fb;
+      } else if (xsrc != nullptr) {
+        lane_bulk(dst + C::CODE + lane * C::XB, xsrc, xbytes, fb);
       }
+#pragma unroll
+      for (int pj = 0; pj < NPROJ; ++pj) {
+        const uint8_t* src = isrc[pj] + atom * kBlk;
+        const uint32_t sdst = dst + C::SC_OFF + pj * C::SC + lane * kBlk;
+        if (whole) {
+#pragma unroll
+          for (int w = 0; w < kBlk; w += 4) lane_cp4(sdst + w, src + w);
+        } else {  // the last atom of a row: nb - atom * kBlk scale bytes, a multiple of 4
+          for (int w = 0; w < nb - atom * kBlk; w += 4) lane_cp4(sdst + w, src + w);
+        }
+      }
+      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(fb) : "memory");
       it_next(nxt, *l, pfx, nV);
       ++jv;
     }
+    else if constexpr (DJ >= 0) {
+      dsrc[DJ] = nullptr;
+    }
+    if (++islot == C::D) islot = 0;
     ++ji;
+  }
+
+  // The deferred token-row copies of the prologue stages.
+  __device__ __forceinline__ void flush_deferred() {
+#pragma unroll
+    for (int j = 0; j < C::D; ++j)
+      if (dsrc[j] != nullptr) lane_bulk(ddst[j], dsrc[j], dbytes[j], dfb[j]);
   }
 
   // After a timeout: let the copies already issued land (bounded) so the
@@ -342,46 +426,24 @@ struct LaneWarp {
         }
       }
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncwarp();
   }
 
-  // Start loading the scale bytes of stage `look` (this lane's row, 8 blocks).
-  __device__ __forceinline__ void load_scales() {
-    if (!look.valid) return;
-    const int atom = look.a - look.blk * l->NA;
-    const int e = expert(look.v);
-    const bool sh = e < 0;
-    const int row = look.rb * 32 + lane;
-#pragma unroll
-    for (int pj = 0; pj < NPROJ; ++pj) {
-      const uint8_t* sbase;
-      if (PHASE == 0)
-        sbase = sh ? (pj == 0 ? a->sh.gs : a->sh.us) : (pj == 0 ? a->ex.gs : a->ex.us);
-      else
-        sbase = sh ? a->sh.ds : a->ex.ds;
-      if (!sh) sbase += size_t(e) * ROWS * nb;
-      const uint8_t* src = sbase + size_t(row) * nb + atom * 8;
-      if ((nb & 7) == 0) {
-        scn[pj] = ldg_na8(src);
-      } else {  // nb % 8 == 4: a 4-byte aligned row; the last atom has 4 bytes
-        scn[pj].x = ldg_na4(src);
-        scn[pj].y = nb - atom * 8 > 4 ? ldg_na4(src + 4) : 0u;
-      }
-    }
-  }
 };
 
 // ---------------------------------------------------------- stage compute ---
 // Phase 0: gate and up rows of the lane, R tokens (the slot's f16 values).
 template <int R>
-__device__ __forceinline__ void stage_gateup(const unsigned char* slot, uint2 sg, uint2 su,
+__device__ __forceinline__ void stage_gateup(const unsigned char* slot, ScaleWord sg, ScaleWord su,
                                              int nblk, int lane, float (&ag)[R], float (&au)[R]) {
   const unsigned char* rg = slot + lane * kAtomCode;
   const unsigned char* ru = slot + kBox + lane * kAtomCode;
   const unsigned char* xs = slot + 2 * kBox;
-  const int sw = lane & 7;
-#pragma unroll 1
-  for (int j = 0; j < nblk; ++j) {
+  const int sw = swz(lane);
+#pragma unroll
+  for (int j = 0; j < kBlk; ++j) {
+    if (kBlk > 4 && j >= nblk) break;
     const uint4 cg = *reinterpret_cast<const uint4*>(rg + ((j ^ sw) << 4));
     const uint4 cu = *reinterpret_cast<const uint4*>(ru + ((j ^ sw) << 4));
     uint32_t wg[16], wu[16];
@@ -397,7 +459,7 @@ __device__ __forceinline__ void stage_gateup(const unsigned char* slot, uint2 sg
     const float fu = e8m0_to_f32(scale_byte(su, j));
 #pragma unroll
     for (int t = 0; t < R; ++t) {
-      const uint4* xp = reinterpret_cast<const uint4*>(xs + t * 512 + j * 64);
+      const uint4* xp = reinterpret_cast<const uint4*>(xs + t * (kAtomVals * 2) + j * 64);
       const uint4 x0 = xp[0], x1 = xp[1], x2 = xp[2], x3 = xp[3];
       const uint32_t xv[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
                                x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
@@ -417,13 +479,14 @@ __device__ __forceinline__ void stage_gateup(const unsigned char* slot, uint2 sg
 
 // Phase 1: down row of the lane, R tokens (the slot's f32 values).
 template <int R>
-__device__ __forceinline__ void stage_down(const unsigned char* slot, uint2 sd, int nblk,
+__device__ __forceinline__ void stage_down(const unsigned char* slot, ScaleWord sd, int nblk,
                                            int lane, float (&ad)[R]) {
   const unsigned char* rd = slot + lane * kAtomCode;
   const unsigned char* xs = slot + kBox;
-  const int sw = lane & 7;
-#pragma unroll 1
-  for (int j = 0; j < nblk; ++j) {
+  const int sw = swz(lane);
+#pragma unroll
+  for (int j = 0; j < kBlk; ++j) {
+    if (kBlk > 4 && j >= nblk) break;
     const uint4 c = *reinterpret_cast<const uint4*>(rd + ((j ^ sw) << 4));
     uint32_t w[16];
     e2m1x8_to_f16x2(c.x, *reinterpret_cast<uint32_t(*)[4]>(&w[0]));
@@ -436,7 +499,7 @@ __device__ __forceinline__ void stage_down(const unsigned char* slot, uint2 sd, 
     const float fd = e8m0_to_f32(scale_byte(sd, j));
 #pragma unroll
     for (int t = 0; t < R; ++t) {
-      const float4* xp = reinterpret_cast<const float4*>(xs + t * 1024 + j * 128);
+      const float4* xp = reinterpret_cast<const float4*>(xs + t * (kAtomVals * 4) + j * 128);
       float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0, s3 = s0;
 #pragma unroll
       for (int q = 0; q < 8; q += 2) {
@@ -485,17 +548,15 @@ __device__ bool run_pass(LaneWarp<PHASE>& W, LaneIt& cur, const VExpert& ve) {
   for (int t = 0; t < R; ++t) acc0[t] = acc1[t] = 0.f;
 
   for (int s = 0; s < nst; ++s) {
-    const int d = W.jc % C::D;
+    const int d = W.cslot;
     const int atom = cur.a - blk * l.NA;
-    const int nblk = min(8, W.nb - atom * 8);
-    // this stage's scale bytes; start loading the next stage's
-    uint2 sc[NPROJ];
-#pragma unroll
-    for (int pj = 0; pj < NPROJ; ++pj) sc[pj] = W.scn[pj];
-    it_next(W.look, l, W.pfx, W.nV);
-    W.load_scales();
-    if (!lane_wait(lsm(&W.full[d]), uint32_t(W.jc / C::D) & 1u, a.err, 410)) return false;
+    if (!lane_wait(lsm(&W.full[d]), W.cpar, a.err, 410)) return false;
     const unsigned char* slot = W.codes + size_t(d) * C::SLOT;
+    ScaleWord sc[NPROJ];
+#pragma unroll
+    for (int pj = 0; pj < NPROJ; ++pj)
+      sc[pj] = *reinterpret_cast<const ScaleWord*>(slot + C::SC_OFF + pj * C::SC + lane * kBlk);
+    const int nblk = min(kBlk, W.nb - atom * kBlk);
     if constexpr (PHASE == 0) {
       stage_gateup<R>(slot, sc[0], sc[1], nblk, lane, acc0, acc1);
     } else {
@@ -503,6 +564,10 @@ __device__ bool run_pass(LaneWarp<PHASE>& W, LaneIt& cur, const VExpert& ve) {
     }
     __syncwarp();
     ++W.jc;
+    if (++W.cslot == C::D) {
+      W.cslot = 0;
+      W.cpar ^= 1u;
+    }
     W.issue();
     it_next(cur, l, W.pfx, W.nV);
   }
@@ -586,11 +651,14 @@ __global__ void __launch_bounds__(kLThreads, 1)
   W.full = bars + warp * C::D;
   if (lane == 0) {
     for (int d = 0; d < C::D; ++d)
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(lsm(&W.full[d])));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 33;" ::"r"(lsm(&W.full[d])));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncwarp();
-  pdl_wait();
+  // The down projection's routing data (plan, buckets) and weights are ready
+  // before the previous kernel (gate/up) ends: its setup and first weight
+  // loads run ahead of the wait; only its token rows (h) wait.
+  if constexpr (PHASE == 0) pdl_wait();
   pdl_trigger();
 
   W.K = PHASE == 0 ? a.H : a.I;
@@ -603,13 +671,18 @@ __global__ void __launch_bounds__(kLThreads, 1)
   W.ev = -1;
   W.ee = -1;
   W.iv = -1;
+  W.ipass = -1;
+  W.iseg = -1;
+  W.islot = W.cslot = 0;
+  W.cpar = 0;
+
 
   // Per virtual expert: tokens, passes and cost; prefix sums over the experts
   // (two entries per thread).
   {
     int* s_cpfx = s_pfx + kPfxMax;
     int* s_rv = s_cpfx + kPfxMax;
-    int* s_wsum = s_rv + kPfxMax;  // [8][2]
+    int* s_wsum = s_rv + kPfxMax;  // [kLW][2]
     const int tid = threadIdx.x;
     int np[2] = {0, 0}, cu[2] = {0, 0};
 #pragma unroll
@@ -667,14 +740,25 @@ __global__ void __launch_bounds__(kLThreads, 1)
   W.gw = blockIdx.x * kLW + warp;
   W.A0 = W.part.atom_at(W.gw);
   W.A1 = W.part.atom_at(W.gw + 1);
-  if (W.A0 >= W.A1) return;
+  if (W.A0 >= W.A1) {
+    if constexpr (PHASE == 1) pdl_wait();
+    return;
+  }
 
   LaneIt cur;
   it_begin(cur, W.A0, W.A1, l, W.pfx, W.nV);
   it_begin(W.nxt, W.A0, W.A1, l, W.pfx, W.nV);
-  for (int d = 0; d < C::D; ++d) W.issue();
-  W.look = cur;
-  W.load_scales();
+  if constexpr (PHASE == 1) {
+    static_assert(C::D <= 4, "prologue");
+    W.template issue<0>();
+    if constexpr (C::D > 1) W.template issue<1>();
+    if constexpr (C::D > 2) W.template issue<2>();
+    if constexpr (C::D > 3) W.template issue<3>();
+    pdl_wait();
+    W.flush_deferred();
+  } else {
+    for (int d = 0; d < C::D; ++d) W.issue();
+  }
 
   int vv = -1;
   VExpert ve{};
@@ -726,13 +810,13 @@ cudaError_t launch_ffn_lane(const FfnArgs& a, float* lane_part, uint32_t* lane_c
   if (!lane_supported(s) || a.xh == nullptr) return cudaErrorNotSupported;
   LaneMaps g{}, d{};
   const uint64_t HB = uint64_t(a.H) / 2, IB = uint64_t(a.I) / 2;
-  bool ok = make_tma_map_u8(&g.m[0], a.ex.gq, HB, uint64_t(a.E) * a.I, 32) &&
-            make_tma_map_u8(&g.m[1], a.ex.uq, HB, uint64_t(a.E) * a.I, 32) &&
-            make_tma_map_u8(&d.m[0], a.ex.dq, IB, uint64_t(a.E) * a.H, 32);
+  bool ok = make_tma_map_u8_box(&g.m[0], a.ex.gq, HB, uint64_t(a.E) * a.I, kAtomCode, 32) &&
+            make_tma_map_u8_box(&g.m[1], a.ex.uq, HB, uint64_t(a.E) * a.I, kAtomCode, 32) &&
+            make_tma_map_u8_box(&d.m[0], a.ex.dq, IB, uint64_t(a.E) * a.H, kAtomCode, 32);
   if (a.has_shared) {
-    ok = ok && make_tma_map_u8(&g.m[2], a.sh.gq, HB, a.I, 32) &&
-         make_tma_map_u8(&g.m[3], a.sh.uq, HB, a.I, 32) &&
-         make_tma_map_u8(&d.m[1], a.sh.dq, IB, a.H, 32);
+    ok = ok && make_tma_map_u8_box(&g.m[2], a.sh.gq, HB, a.I, kAtomCode, 32) &&
+         make_tma_map_u8_box(&g.m[3], a.sh.uq, HB, a.I, kAtomCode, 32) &&
+         make_tma_map_u8_box(&d.m[1], a.sh.dq, IB, a.H, kAtomCode, 32);
   } else {
     g.m[2] = g.m[0];
     g.m[3] = g.m[1];

@@ -20,8 +20,14 @@ constexpr unsigned kFull = 0xffffffffu;
 // GEMV), CTAs (one per SM, at most), warps per CTA, tokens per pass.
 constexpr int kLaneMaxT = 64;
 constexpr int kLaneMaxCtas = 160;
-constexpr int kLaneWarps = 8;
-constexpr int kLaneRMax = 8;
+#ifndef MOE_LANE_WARPS
+#define MOE_LANE_WARPS 11
+#endif
+#ifndef MOE_LANE_RMAX
+#define MOE_LANE_RMAX 8
+#endif
+constexpr int kLaneWarps = MOE_LANE_WARPS;
+constexpr int kLaneRMax = MOE_LANE_RMAX;
 
 // ---------------------------------------------------------------------------
 // Workspace layout.  Every region starts on a 256-byte boundary.
@@ -75,7 +81,8 @@ inline WsLayout ws_layout(const moe_shape_t& s, int has_shared, int gemm) {
   L.lane_part = take(lane ? size_t(kLaneMaxCtas) * kLaneWarps * 2 * kLaneRMax * 2 * 32 * 4 : 0);
   // passes: at most one per virtual expert plus one per kLaneRMax rows
   const size_t passes = E + 1 + (rows + kLaneRMax - 1) / kLaneRMax;
-  const size_t rb0 = I / 32, na0 = (H + 255) / 256, rb1 = H / 32, na1 = (I + 255) / 256;
+  // atoms of at least 128 values
+  const size_t rb0 = I / 32, na0 = (H + 127) / 128, rb1 = H / 32, na1 = (I + 127) / 128;
   L.lane_cnt = take(lane ? passes * (rb0 > rb1 ? rb0 : rb1) * 4 : 0);
   L.lane_tab = take(lane ? passes * (rb0 * na0 > rb1 * na1 ? rb0 * na0 : rb1 * na1) * 4 : 0);
   if (gemm) {
