@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--path", choices=["auto", "gemv", "gemm"], default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="the multi-layer cold-cache batch sweep: GEMV and GEMM paths per T, "
+                         "and the crossover (prints its own JSON line)")
     a = ap.parse_args()
     a.warmup = max(3, a.warmup)
     return a
@@ -277,8 +280,8 @@ def run_ours(args, rank, world, local_rank):
     achieved = ffn_b / (ffn_ms / 1e3) / 1e9
     flops = 6.0 * cfg.H * cfg.I * T * (cfg.k + (1 if cfg.shared else 0))
     tflops = flops / (ffn_ms / 1e3) / 1e12
-    uses_tc = PREC == moe.MOE_ACT_MXFP4 and (
-        PATH == moe.MOE_PATH_GEMM or (PATH == moe.MOE_PATH_AUTO and T * cfg.k >= 512))
+    # AUTO takes the tensor-core kernels for MXFP4 activations at every batch size
+    uses_tc = PREC == moe.MOE_ACT_MXFP4 and PATH in (moe.MOE_PATH_GEMM, moe.MOE_PATH_AUTO)
     fp4_peak = peaks["bf16_tflops"] * 4.0  # dense FP4 = 4 x dense bf16 (nominal ratio)
     t_hbm = ffn_b / (peaks["hbm_gbs"] * 1e9)
     t_tc = flops / (fp4_peak * 1e12)
@@ -407,6 +410,100 @@ def run_extra(cfg, layers, Wd, bd, stream, dev, args):
     return res
 
 
+# ----------------------------------------------------- batch-size sweep ----
+def run_sweep(args, local_rank):
+    """Eight independent copies of the fine-grained layer (Zipf 1.2 routing),
+    called in turn so every call reads cold weights; for each batch size the
+    CUDA-core path (exact and MXFP4 activations) and the tensor-core path
+    (MXFP4 activations) are timed as whole layers.  The crossover is the
+    smallest batch at which the tensor-core path beats the CUDA-core path at
+    the same precision."""
+    import torch
+    from routed_expert_ffn_fp32_b200 import build, moe, synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    build.build()
+    moe.load_library()
+    base = synth.SWEEP
+    NL = synth.SWEEP_LAYERS
+    L = synth.layer(base, seed=0)
+    ex0 = moe.Experts.from_numpy(L["experts"], dev)
+    sh0 = moe.Experts.from_numpy(L["shared"], dev)
+    fields = ("gate_q", "gate_s", "up_q", "up_s", "down_q", "down_s")
+    layers = [(ex0, sh0)] + [
+        (moe.Experts(**{f: getattr(ex0, f).clone() for f in fields}),
+         moe.Experts(**{f: getattr(sh0, f).clone() for f in fields})) for _ in range(NL - 1)]
+    Wd = torch.from_numpy(L["W_r"]).to(dev)
+    bd = torch.from_numpy(L["bias"]).to(dev)
+    stream = torch.cuda.Stream(dev)
+    variants = [("gemv_exact", moe.MOE_PATH_GEMV, moe.MOE_ACT_EXACT),
+                ("gemv_mxfp4", moe.MOE_PATH_GEMV, moe.MOE_ACT_MXFP4),
+                ("gemm_mxfp4", moe.MOE_PATH_GEMM, moe.MOE_ACT_MXFP4)]
+    rows = []
+    for T in synth.SWEEP_T:
+        cfg = base.with_T(T)
+        shape = moe.shape_of(T, cfg.H, cfg.I, cfg.E, cfg.k)
+        NX = 4
+        xs = [torch.from_numpy(synth.activations(cfg, 9000 + i, T).view(np.int16)).to(dev)
+              for i in range(NX)]
+        y = torch.empty((T, cfg.H), dtype=torch.int16, device=dev)
+        idx = torch.empty((T, cfg.k), dtype=torch.int32, device=dev)
+        wts = torch.empty((T, cfg.k), dtype=torch.float32, device=dev)
+        row = {"T": T}
+        nbytes = []
+        for name, path, prec in variants:
+            ws = moe.make_workspace(shape, path, prec, True, dev, stream)
+            ncyc = int(np.lcm(NL, NX))
+            graphs = []
+            with torch.cuda.stream(stream):
+                for i in range(ncyc):
+                    ex, sh = layers[i % NL]
+                    moe.moe_layer_forward(xs[i % NX], Wd, bd, ex, sh, shape, y, ws, path, prec,
+                                          idx, wts, stream=stream)
+                    if name == "gemv_exact":
+                        stream.synchronize()
+                        nbytes.append(activated_bytes(
+                            cfg, np.bincount(idx.cpu().numpy().reshape(-1), minlength=cfg.E)))
+                stream.synchronize()
+                for i in range(ncyc):
+                    ex, sh = layers[i % NL]
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=stream):
+                        moe.moe_layer_forward(xs[i % NX], Wd, bd, ex, sh, shape, y, ws, path,
+                                              prec, idx, wts, stream=stream)
+                    graphs.append(g)
+                for i in range(max(args.warmup, 3)):
+                    graphs[i % ncyc].replay()
+                stream.synchronize()
+                n = max(ncyc, min(200, int(2e5 / T)))
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for i in range(n):
+                    graphs[i % ncyc].replay()
+                b.record(stream)
+                stream.synchronize()
+            assert moe.moe_get_error(ws, stream) == 0
+            ms = a.elapsed_time(b) / n
+            row[name] = {"tokens_per_s": round(T / (ms / 1e3), 1), "ms_per_step": round(ms, 5)}
+            del graphs, ws
+        act = float(np.mean(nbytes))
+        row["activated_bytes_per_call"] = int(act)
+        for name, _, _ in variants:
+            row[name]["hbm_gbs"] = round(act / (row[name]["ms_per_step"] / 1e3) / 1e9, 1)
+        rows.append(row)
+    cross = next((r["T"] for r in rows
+                  if r["gemm_mxfp4"]["tokens_per_s"] > r["gemv_mxfp4"]["tokens_per_s"]), None)
+    peaks = load_peaks()
+    return {"metric": "MoE layer tokens/s over the batch sweep (cold weights, 8 layers)",
+            "unit": "tokens/s", "n_gpus": 1, "data": "synthetic",
+            "config": {"workload": base.name, "layers": NL, "T": list(synth.SWEEP_T),
+                       "weights_gb": round(NL * (cfg.E + 1) * expert_bytes(cfg) / 1e9, 2)},
+            "hbm_peak_gbs": peaks["hbm_gbs"], "sweep": rows,
+            "crossover_T_gemm_over_gemv_mxfp4": cross}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -487,6 +584,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.sweep:
+        if rank == 0:
+            print(json.dumps(run_sweep(args, local_rank)), flush=True)
+        return
     if args.impl == "reference":
         out = run_reference(args, rank, world)
         if out is not None:

@@ -105,9 +105,10 @@ typedef struct moe_mxfp4_experts {
   int32_t n_experts;
 } moe_mxfp4_experts_t;
 
-/* Expert FFN implementation.  GEMV: CUDA-core streaming kernels, exact bf16
- * activations (decode / verify).  GEMM: tcgen05 block-scaled FP4 tensor-core
- * kernels (prefill), which require MOE_ACT_MXFP4.  AUTO picks by batch size. */
+/* Expert FFN implementation.  GEMV: CUDA-core streaming kernels (either
+ * precision).  GEMM: tcgen05 block-scaled FP4 tensor-core kernels, which
+ * require MOE_ACT_MXFP4.  AUTO: GEMM for MOE_ACT_MXFP4 (when the shape allows
+ * it: H % 256 == 0, I % 128 == 0), GEMV for MOE_ACT_EXACT. */
 #define MOE_PATH_AUTO 0
 #define MOE_PATH_GEMV 1
 #define MOE_PATH_GEMM 2

@@ -18,7 +18,7 @@ constexpr int kMaxTopK = 16;
 constexpr unsigned kFull = 0xffffffffu;
 // Lane-per-row GEMV: largest batch it takes (larger ones use the K-split
 // GEMV), CTAs (one per SM, at most), warps per CTA, tokens per pass.
-constexpr int kLaneMaxT = 64;
+constexpr int kLaneMaxT = 512;
 constexpr int kLaneMaxCtas = 160;
 #ifndef MOE_LANE_WARPS
 #define MOE_LANE_WARPS 11
