@@ -121,6 +121,23 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(inside)}
 
 
+# ------------------------------------------------------------ ranks -------
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest value over all ranks (step time is max over ranks); dist is
+    torch.distributed or None for one process."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(tokens_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job tokens/s: every rank runs its own batches of the same size."""
+    return world * tokens_per_rank / (ms / 1e3)
+
+
 # ------------------------------------------------------------- workload ----
 def workload(name: str, T: int):
     from routed_expert_ffn_fp32_b200 import synth
@@ -233,13 +250,9 @@ def run_ours(args, rank, world, local_rank):
         barrier()
     sampler.stop()
     ms_local = e0.elapsed_time(e1) / args.steps
-    ms = ms_local
-    if dist is not None:
-        t = torch.tensor([ms_local], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms_local, dist, dev)
     assert moe.moe_get_error(ws, stream) == 0
-    value = world * T / (ms / 1e3)
+    value = weak_scaling_value(T, world, ms)
 
     # ---- dominant kernels: expert FFN (gate/up + down) timed alone -------------
     offs = torch.empty(cfg.E + 1, dtype=torch.int32, device=dev)
