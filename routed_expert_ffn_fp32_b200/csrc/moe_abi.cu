@@ -301,7 +301,11 @@ moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router, const f
   if (rp == MOE_PATH_GEMV) {
     r.xh = at<uint16_t>(ws, L.xh);
     r.act_mxfp4 = precision == MOE_ACT_MXFP4;
+    // the fused router tail also writes the lane GEMV's per-expert tables
+    if (shape.T <= kFusedRouteMaxT && lane_supported(shape))
+      r.lane_pre = at<int32_t>(ws, L.lane_pre);
   }
+  r.has_shared = has_shared;
   cudaError_t e;
   if (shape.T <= kFusedRouteMaxT) {
     e = launch_route_logits(r, true, s);
@@ -332,6 +336,7 @@ moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router, const f
   a.has_shared = has_shared;
   a.act_mxfp4 = precision == MOE_ACT_MXFP4;
   a.xh = r.xh;
+  a.lane_pre = r.lane_pre;
   e = rp == MOE_PATH_GEMM ? launch_ffn_gemm(a, gemm_buffers(ws, L, shape.E), s)
                           : launch_gemv_path(a, ws, L, s);
   if (e == cudaSuccess)

@@ -75,7 +75,7 @@ __device__ __forceinline__ int swz(int lane) {
 }
 constexpr unsigned long long kLWaitNs = 2000000000ull;
 
-constexpr int kPfxMax = 258;             // per-expert table entries (virtual experts + 1)
+constexpr int kPfxMax = kLanePfxMax;     // per-expert table entries (virtual experts + 1)
 
 // Shared memory: [barriers][pass prefix][cost prefix][tokens][scan scratch],
 // then the slots from the next 1024-byte boundary.
@@ -678,8 +678,16 @@ __global__ void __launch_bounds__(kLThreads, 1)
 
 
   // Per virtual expert: tokens, passes and cost; prefix sums over the experts
-  // (two entries per thread).
-  {
+  // (two entries per thread), or the same tables as the fused router tail
+  // wrote them.
+  if (a.lane_pre != nullptr) {
+    for (int i = threadIdx.x; i <= W.nV; i += blockDim.x) {
+      s_pfx[i] = __ldg(a.lane_pre + kPfxMax + i);
+      s_pfx[kPfxMax + i] = __ldg(a.lane_pre + 2 * kPfxMax + i);
+      s_pfx[2 * kPfxMax + i] = __ldg(a.lane_pre + i);
+    }
+    __syncthreads();
+  } else {
     int* s_cpfx = s_pfx + kPfxMax;
     int* s_rv = s_cpfx + kPfxMax;
     int* s_wsum = s_rv + kPfxMax;  // [kLW][2]
@@ -726,6 +734,10 @@ __global__ void __launch_bounds__(kLThreads, 1)
       ec += cu[i];
     }
     __syncthreads();
+  }
+  {
+    int* s_cpfx = s_pfx + kPfxMax;
+    int* s_rv = s_cpfx + kPfxMax;
     W.pfx = s_pfx;
     W.part.pfx = s_pfx;
     W.part.cpfx = s_cpfx;

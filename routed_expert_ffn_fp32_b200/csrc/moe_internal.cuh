@@ -28,6 +28,9 @@ constexpr int kLaneMaxCtas = 160;
 #endif
 constexpr int kLaneWarps = MOE_LANE_WARPS;
 constexpr int kLaneRMax = MOE_LANE_RMAX;
+// Per-virtual-expert tables of the lane GEMV's work split (tokens, passes
+// before v, cost units before v), [3][kLanePfxMax]: virtual experts + 1.
+constexpr int kLanePfxMax = 258;
 
 // ---------------------------------------------------------------------------
 // Workspace layout.  Every region starts on a 256-byte boundary.
@@ -49,6 +52,7 @@ struct WsLayout {
   size_t lane_part;  // f32 [warps][2][kLaneRMax][2][32]  split row-block partial sums
   size_t lane_cnt;   // u32 [row blocks]  split row-block arrivals  } zero between calls;
   size_t lane_tab;   // i32 [row blocks][atoms]  contributors   } each call leaves them zero
+  size_t lane_pre;   // i32 [3][kLanePfxMax]  per-expert tables of the work split
   // tensor-core path only
   size_t xq, xs;    // u8 [rows, H/2], [rows, H/32]  MXFP4 token rows, bucket order
   size_t hq, hs;    // u8 [rows, I/2], [rows, I/32]  MXFP4 SwiGLU rows, bucket order
@@ -85,6 +89,7 @@ inline WsLayout ws_layout(const moe_shape_t& s, int has_shared, int gemm) {
   const size_t rb0 = I / 32, na0 = (H + 127) / 128, rb1 = H / 32, na1 = (I + 127) / 128;
   L.lane_cnt = take(lane ? passes * (rb0 > rb1 ? rb0 : rb1) * 4 : 0);
   L.lane_tab = take(lane ? passes * (rb0 * na0 > rb1 * na1 ? rb0 * na0 : rb1 * na1) * 4 : 0);
+  L.lane_pre = take(lane ? 3 * kLanePfxMax * 4 : 0);
   if (gemm) {
     L.xq = take(rows * H / 2);
     L.xs = take(rows * H / 32);
@@ -277,6 +282,8 @@ struct RouteArgs {
   int32_t* plan;
   uint32_t* counter;
   int* err;
+  int32_t* lane_pre;  // optional: the lane GEMV's per-expert tables, written by the fused tail
+  int has_shared;
   int T, H, E, k;
 };
 
@@ -296,6 +303,7 @@ struct FfnArgs {
   int T, H, I, E, k;
   int has_shared;
   int act_mxfp4;
+  const int32_t* lane_pre;  // lane GEMV tables from the fused router tail, or nullptr
 };
 
 // ---------------------------------------------------------------------------
