@@ -102,13 +102,13 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<unsigned char*>(ws) + off);
 }
 
-// CUDA-core FFN: the lane-per-row GEMV where the shape fits it, else the
+// CUDA-core FFN: the row-block mma.sync GEMV where the shape fits it, else the
 // K-split GEMV.
 cudaError_t launch_gemv_path(const FfnArgs& a, void* ws, const WsLayout& L, cudaStream_t s) {
   const moe_shape_t shape{a.T, a.H, a.I, a.E, a.k};
   if (a.xh != nullptr && lane_supported(shape)) {
-    const cudaError_t e = launch_ffn_lane(a, at<float>(ws, L.lane_part),
-                                          at<uint32_t>(ws, L.lane_cnt), at<int>(ws, L.lane_tab), s);
+    const cudaError_t e =
+        launch_ffn_lane(a, at<float>(ws, L.lane_part), at<uint32_t>(ws, L.lane_cnt), s);
     if (e != cudaErrorNotSupported) return e;
   }
   return launch_ffn_gemv(a, s);
@@ -301,9 +301,6 @@ moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router, const f
   if (rp == MOE_PATH_GEMV) {
     r.xh = at<uint16_t>(ws, L.xh);
     r.act_mxfp4 = precision == MOE_ACT_MXFP4;
-    // the fused router tail also writes the lane GEMV's per-expert tables
-    if (shape.T <= kFusedRouteMaxT && lane_supported(shape))
-      r.lane_pre = at<int32_t>(ws, L.lane_pre);
   }
   r.has_shared = has_shared;
   cudaError_t e;
@@ -336,7 +333,6 @@ moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router, const f
   a.has_shared = has_shared;
   a.act_mxfp4 = precision == MOE_ACT_MXFP4;
   a.xh = r.xh;
-  a.lane_pre = r.lane_pre;
   e = rp == MOE_PATH_GEMM ? launch_ffn_gemm(a, gemm_buffers(ws, L, shape.E), s)
                           : launch_gemv_path(a, ws, L, s);
   if (e == cudaSuccess)

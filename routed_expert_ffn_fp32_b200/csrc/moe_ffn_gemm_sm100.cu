@@ -720,7 +720,7 @@ cudaError_t launch_gemm_phase(const GemmArgs& g, const CUtensorMap& a0, const CU
 }  // namespace
 
 // 2-D map of a [rows, row_bytes] uint8 matrix, boxes of box_rows x box_bytes
-// (64 or 128) with the swizzle of the same width (the lane-per-row GEMV's
+// (64 or 128) with the swizzle of the same width (the decode GEMV's
 // code boxes).
 bool make_tma_map_u8_box(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
                          uint32_t box_bytes, uint32_t box_rows) {
@@ -733,6 +733,21 @@ bool make_tma_map_u8_box(CUtensorMap* m, const void* base, uint64_t row_bytes, u
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE,
             box_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map of a [rows, row_bytes] uint8 matrix (row_bytes a multiple of 16),
+// boxes of box_rows x box_bytes, no swizzle (the decode GEMV's scale boxes).
+bool make_tma_map_u8_plain(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
+                           uint32_t box_bytes, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr || row_bytes % 16 != 0 || box_bytes % 16 != 0) return false;
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_bytes, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

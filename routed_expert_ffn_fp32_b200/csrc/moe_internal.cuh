@@ -16,7 +16,7 @@ namespace moe {
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 16;
 constexpr unsigned kFull = 0xffffffffu;
-// Lane-per-row GEMV: largest batch it takes (larger ones use the K-split
+// Row-block mma.sync GEMV: largest batch it takes (larger ones use the K-split
 // GEMV), CTAs (one per SM, at most), warps per CTA, tokens per pass.
 constexpr int kLaneMaxT = 512;
 constexpr int kLaneMaxCtas = 160;
@@ -28,8 +28,8 @@ constexpr int kLaneMaxCtas = 160;
 #endif
 constexpr int kLaneWarps = MOE_LANE_WARPS;
 constexpr int kLaneRMax = MOE_LANE_RMAX;
-// Per-virtual-expert tables of the lane GEMV's work split (tokens, passes
-// before v, cost units before v), [3][kLanePfxMax]: virtual experts + 1.
+// Per-virtual-expert tables of the row-block GEMV's work split (tokens, passes
+// before v, cost units before v, plan, offsets): virtual experts + 1 entries.
 constexpr int kLanePfxMax = 258;
 
 // ---------------------------------------------------------------------------
@@ -46,13 +46,12 @@ struct WsLayout {
   size_t entries;   // i32 [T * k]
   size_t plan;      // i32 [E + 2]: [0] active experts, [1..] their ids (ascending)
   size_t xh;        // f16 [T, H]  token rows as f16 (MXFP4-rounded in that mode)
-  size_t h;         // f32 [T*k + S*T, I]   SwiGLU output rows (by pair index)
+  size_t h;         // [T*k + S*T] rows of 4I bytes: SwiGLU output by pair index (f32, or f16 hi then f16 lo in the row-block GEMV)
   size_t partial;   // f32 [T*k + S*T, H]   expert output rows (by pair index)
-  // lane-per-row GEMV (T <= kLaneMaxT)
-  size_t lane_part;  // f32 [warps][2][kLaneRMax][2][32]  split row-block partial sums
-  size_t lane_cnt;   // u32 [row blocks]  split row-block arrivals  } zero between calls;
-  size_t lane_tab;   // i32 [row blocks][atoms]  contributors   } each call leaves them zero
-  size_t lane_pre;   // i32 [3][kLanePfxMax]  per-expert tables of the work split
+  // row-block GEMV (T <= kLaneMaxT)
+  size_t lane_part;  // f32 [warps][kLaneRMax][2][32]  split row-block partial sums
+  size_t lane_cnt;   // u32 [row blocks]  split row-block atom counts: zero between calls,
+                     //     every call leaves them zero
   // tensor-core path only
   size_t xq, xs;    // u8 [rows, H/2], [rows, H/32]  MXFP4 token rows, bucket order
   size_t hq, hs;    // u8 [rows, I/2], [rows, I/32]  MXFP4 SwiGLU rows, bucket order
@@ -82,14 +81,11 @@ inline WsLayout ws_layout(const moe_shape_t& s, int has_shared, int gemm) {
   L.h = take(rows * I * 4);
   L.partial = take(rows * H * 4);
   const bool lane = T <= size_t(kLaneMaxT);
-  L.lane_part = take(lane ? size_t(kLaneMaxCtas) * kLaneWarps * 2 * kLaneRMax * 2 * 32 * 4 : 0);
+  L.lane_part = take(lane ? size_t(kLaneMaxCtas) * kLaneWarps * kLaneRMax * 2 * 32 * 4 : 0);
   // passes: at most one per virtual expert plus one per kLaneRMax rows
   const size_t passes = E + 1 + (rows + kLaneRMax - 1) / kLaneRMax;
-  // atoms of at least 128 values
-  const size_t rb0 = I / 32, na0 = (H + 127) / 128, rb1 = H / 32, na1 = (I + 127) / 128;
+  const size_t rb0 = I / 32, rb1 = H / 32;  // row blocks of the two phases
   L.lane_cnt = take(lane ? passes * (rb0 > rb1 ? rb0 : rb1) * 4 : 0);
-  L.lane_tab = take(lane ? passes * (rb0 * na0 > rb1 * na1 ? rb0 * na0 : rb1 * na1) * 4 : 0);
-  L.lane_pre = take(lane ? 3 * kLanePfxMax * 4 : 0);
   if (gemm) {
     L.xq = take(rows * H / 2);
     L.xs = take(rows * H / 32);
@@ -282,7 +278,6 @@ struct RouteArgs {
   int32_t* plan;
   uint32_t* counter;
   int* err;
-  int32_t* lane_pre;  // optional: the lane GEMV's per-expert tables, written by the fused tail
   int has_shared;
   int T, H, E, k;
 };
@@ -303,7 +298,6 @@ struct FfnArgs {
   int T, H, I, E, k;
   int has_shared;
   int act_mxfp4;
-  const int32_t* lane_pre;  // lane GEMV tables from the fused router tail, or nullptr
 };
 
 // ---------------------------------------------------------------------------
@@ -375,7 +369,7 @@ cudaError_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t st);
 // Lane-per-row GEMV of both phases; cudaErrorNotSupported when the shape does
 // not fit it (the caller then uses launch_ffn_gemv).
 cudaError_t launch_ffn_lane(const FfnArgs& a, float* lane_part, uint32_t* lane_cnt,
-                            int* lane_tab, cudaStream_t st);
+                            cudaStream_t st);
 bool lane_supported(const moe_shape_t& s);
 cudaError_t launch_x_f16(const uint16_t* x, int T, int H, int act_mxfp4, uint16_t* xh,
                          cudaStream_t st);

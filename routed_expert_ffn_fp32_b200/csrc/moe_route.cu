@@ -15,7 +15,7 @@
 //     warp w takes expert (w / 4) of the pair and the w % 4 quarter of H; each
 //     lane streams float4 router rows and keeps TT float32 partial sums.  The
 //     bf16 token rows sit in shared memory; the f16 copy of the token rows
-//     for the lane GEMV is written from there by all CTAs of a token tile,
+//     for the row-block GEMV is written from there by all CTAs of a token tile,
 //     32 values per thread.  Every product meets at most
 //     H/128 + 9 roundings (lane chain, 5 shuffle levels, 3 quarter sums, the
 //     bias), the bound the parity tests use for near-ties.
@@ -261,7 +261,7 @@ __device__ void bucket_block(const int32_t* idx, int npairs, int E, int32_t* cou
 // order, ranks among equal experts from __match_any_sync.  No block barrier.
 __device__ int bucket_warp(const int32_t* idx, int npairs, int E, int32_t* counts,
                            int32_t* offsets, int32_t* entries, int32_t* plan, int* err, int* cnt,
-                           int* cur, int32_t* rv) {
+                           int* cur) {
   const int lane = threadIdx.x & 31;
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int e = lane; e < E; e += 32) cnt[e] = 0;
@@ -291,10 +291,7 @@ __device__ int bucket_warp(const int32_t* idx, int npairs, int E, int32_t* count
       counts[e] = c;
       offsets[e] = ex;
       cur[e] = ex;
-      if (act) {
-        plan[1 + run_act + incl_act - 1] = e;
-        if (rv) rv[run_act + incl_act - 1] = c;
-      }
+      if (act) plan[1 + run_act + incl_act - 1] = e;
     }
     run += __shfl_sync(kFull, incl, 31);
     run_act += __shfl_sync(kFull, incl_act, 31);
@@ -316,37 +313,6 @@ __device__ int bucket_warp(const int32_t* idx, int npairs, int E, int32_t* count
     __syncwarp();
   }
   return run_act;
-}
-
-// The lane GEMV's per-virtual-expert tables (one warp): tokens R_v (the
-// routed counts already in rv, then T for the shared expert), passes of at
-// most kLaneRMax tokens before v, and cost units (passes + tokens) before v.
-__device__ void lane_tables_warp(int32_t* pre, int nA, int has_shared, int T) {
-  const int lane = threadIdx.x & 31;
-  const int nV = nA + (has_shared ? 1 : 0);
-  if (has_shared && lane == 0) pre[nA] = T;
-  __syncwarp();
-  int run_p = 0, run_c = 0;
-  for (int base = 0; base <= nV; base += 32) {
-    const int v = base + lane;
-    const int R = v < nV ? pre[v] : 0;
-    const int np = (R + kLaneRMax - 1) / kLaneRMax, cu = np + R;
-    int ip = np, ic = cu;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int yp = __shfl_up_sync(kFull, ip, off), yc = __shfl_up_sync(kFull, ic, off);
-      if (lane >= off) {
-        ip += yp;
-        ic += yc;
-      }
-    }
-    if (v <= nV) {
-      pre[kLanePfxMax + v] = run_p + ip - np;
-      pre[2 * kLanePfxMax + v] = run_c + ic - cu;
-    }
-    run_p += __shfl_sync(kFull, ip, 31);
-    run_c += __shfl_sync(kFull, ic, 31);
-  }
 }
 
 // ---------------------------------------------------------------- kernels ---
@@ -452,9 +418,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_logits(RouteArgs a, int
   __syncthreads();
   if (warp == 0) {
     int* cnt = reinterpret_cast<int*>(smem + align_up16(size_t(a.T) * a.k * 4));
-    const int nA = bucket_warp(idx_s, a.T * a.k, a.E, a.counts, a.offsets, a.entries, a.plan,
-                               a.err, cnt, cnt + a.E, a.lane_pre);
-    if (a.lane_pre != nullptr) lane_tables_warp(a.lane_pre, nA, a.has_shared, a.T);
+    bucket_warp(idx_s, a.T * a.k, a.E, a.counts, a.offsets, a.entries, a.plan, a.err, cnt,
+                cnt + a.E);
     if (lane == 0) *a.counter = 0u;
   }
 }
