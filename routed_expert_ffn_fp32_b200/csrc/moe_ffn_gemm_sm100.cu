@@ -147,6 +147,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
+// The same with an L2 cache policy (expert weights: read once per call,
+// evict first, so they do not push the activations, the router weights and
+// the workspace out of L2).
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                                 uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+      : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -390,10 +401,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       unsigned char* sfb = sfa + NPROJ * C::SFA_BYTES;
       const uint32_t fb = saddr(&full[stage]);
       if (lane == 0) {
+        uint64_t pol;
+        asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
         mbar_expect_tx(fb, NPROJ * C::A_BYTES + C::B_BYTES);
-        tma_load_2d(saddr(st), routed ? &mA0 : &mS0, ks * kBKB, arow, fb);
+        tma_load_2d_hint(saddr(st), routed ? &mA0 : &mS0, ks * kBKB, arow, fb, pol);
         if constexpr (NPROJ == 2)
-          tma_load_2d(saddr(st + C::A_BYTES), routed ? &mA1 : &mS1, ks * kBKB, arow, fb);
+          tma_load_2d_hint(saddr(st + C::A_BYTES), routed ? &mA1 : &mS1, ks * kBKB, arow, fb, pol);
         tma_load_2d(saddr(st + NPROJ * C::A_BYTES), &mB, ks * kBKB, brow, fb);
       }
       // scale words -> atom layout: K atom `at` of row r at at*512 + 16*(r%32) + 4*(r/32%4)

@@ -170,6 +170,21 @@ __device__ __forceinline__ void lane_tma(uint32_t dst, const CUtensorMap* map, i
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
+// The same with an L2 cache policy (weights: read once, evict first, so the
+// stream does not push out the instructions and the small hot data).
+__device__ __forceinline__ void lane_tma_hint(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                              uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
 __device__ __forceinline__ void lane_cp4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -431,13 +446,14 @@ struct LaneWarp {
                      "r"(uint32_t(NPROJ * kBox) + uint32_t(irows) * kXRow +
                          (sload ? uint32_t(C::SCE) : 0u))
                      : "memory");
+        const uint64_t pol = evict_first_policy();
 #pragma unroll
         for (int pj = 0; pj < NPROJ; ++pj)
-          lane_tma(dst + pj * kBox, imap + pj, atom * kAtomCode, iy, fb);
+          lane_tma_hint(dst + pj * kBox, imap + pj, atom * kAtomCode, iy, fb, pol);
         if (sload)
 #pragma unroll
           for (int pj = 0; pj < NPROJ; ++pj)
-            lane_tma(sdst + pj * (C::SCE / NPROJ), ismap + pj, 16 * (atom >> 2), iy, fb);
+            lane_tma_hint(sdst + pj * (C::SCE / NPROJ), ismap + pj, 16 * (atom >> 2), iy, fb, pol);
       }
       __syncwarp();
       const void* xsrc = lane < irows ? ixsrc + size_t(kbase) * 2 : nullptr;
