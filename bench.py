@@ -300,9 +300,13 @@ def run_ours(args, rank, world, local_rank):
     t_tc = flops / (fp4_peak * 1e12)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": None, "kernel": "expert FFN (gate/up + SwiGLU, down)",
+                "traffic": None, "kernel": "expert FFN call (plan, f16 token rows, gate/up + SwiGLU, down)",
                 "peak_source": peaks["source"], "bytes_per_launch": int(ffn_b),
                 "launch_ms": round(ffn_ms, 5)}
+    if not uses_tc and cfg.T <= 512:
+        roofline["traffic"] = measured_traffic(ffn_b)
+        roofline["traffic_source"] = "ncu dram__bytes_read.sum + dram__bytes_write.sum of k_ffn_mma " \
+                                     "(profiles/k_ffn_mma_decode64_t5.json), scaled by activated bytes"
     if uses_tc:
         roofline["kernel"] = "expert FFN on tcgen05 kind::mxf4 (gate/up + SwiGLU + requant, down)"
         roofline["tensor"] = {
@@ -515,6 +519,22 @@ def run_sweep(args, local_rank):
                        "weights_gb": round(NL * (cfg.E + 1) * expert_bytes(cfg) / 1e9, 2)},
             "hbm_peak_gbs": peaks["hbm_gbs"], "sweep": rows,
             "crossover_T_gemm_over_gemv_mxfp4": cross}
+
+
+def measured_traffic(bytes_per_launch: float):
+    """DRAM bytes per FFN call from the committed ncu record of the decode GEMV,
+    scaled by the activated bytes of this workload (traffic grows with them);
+    None once the kernel source has changed since the counters were taken, or
+    for another kernel."""
+    import hashlib
+    rec = os.path.join(ROOT, "profiles", "k_ffn_mma_decode64_t5.json")
+    if not os.path.exists(rec):
+        return None
+    d = json.load(open(rec))
+    src = os.path.join(ROOT, d["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != d["source_sha256"]:
+        return None
+    return int(d["dram_bytes_per_call"] / d["algorithmic_bytes_per_call"] * bytes_per_launch)
 
 
 def load_peaks():

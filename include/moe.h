@@ -114,12 +114,16 @@ typedef struct moe_mxfp4_experts {
 #define MOE_PATH_GEMM 2
 
 /* Activation precision of the expert projections.  EXACT: the bf16 token
- * rows and the fp32 SwiGLU output enter the projections as they are (the
- * pages' quality mode, "ds4-ssd" README, "Experimental Pro Support":
- * --quality / --no-int8).  MXFP4: each projection input row is quantised to
- * MXFP4 in 32-element blocks first (scale 2^(floor(log2 amax) - 2),
- * round-to-nearest-even onto the E2M1 grid, saturating at +-6), as an
- * accelerator path does. */
+ * rows and the fp32 SwiGLU output enter the projections without quantisation
+ * (the pages' quality mode, "ds4-ssd" README, "Experimental Pro Support":
+ * --quality / --no-int8), with float32 accumulation.  On the CUDA-core path
+ * for T <= 512 (the row-block GEMV, whose products run on f16 tensor-core
+ * operands) the tokens enter as f16 (exact for 2^-17 <= |x| < 65520) and the
+ * SwiGLU output h as the pair hi = f16(h), lo = f16(h - hi) (22 significant
+ * bits); an |h| of 65520 or more latches MOE_ERR_DEVICE_DATA.  MXFP4: each
+ * projection input row is quantised to MXFP4 in 32-element blocks first
+ * (scale 2^(floor(log2 amax) - 2), round-to-nearest-even onto the E2M1 grid,
+ * saturating at +-6), as an accelerator path does. */
 #define MOE_ACT_EXACT 0
 #define MOE_ACT_MXFP4 1
 

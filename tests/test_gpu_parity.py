@@ -232,6 +232,24 @@ def test_layer_edge_shapes(H, I, E, k, T, shared, bias):
     assert rel_l2(O.bf16_bits_to_f64(out["y"]), O.bf16_bits_to_f64(ref["y_bf16"])) < TOL_Y
 
 
+def test_h_beyond_f16_range_latches_device_data():
+    """The row-block GEMV carries the SwiGLU output to the down projection as
+    an f16 pair: an |h| that f16 cannot hold must latch an error, not turn
+    into infinities.  Every weight 6 * 2^13 and x = 1 give |g|, |u| ~ 1.3e7."""
+    cfg = synth.TINY
+    L = synth.layer(cfg, 0)
+    L["experts"] = {n: (np.full_like(a, 0x77) if n.endswith("_q") else np.full_like(a, 140))
+                    for n, a in L["experts"].items()}
+    L["x"] = np.full_like(L["x"], 0x3F80)   # bf16 1.0
+    D = dev_layer(L)
+    shape = moe.shape_of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k)
+    ws = moe.make_workspace(shape, moe.MOE_PATH_GEMV)
+    y = torch.empty((cfg.T, cfg.H), dtype=torch.int16, device="cuda")
+    moe.moe_layer_forward(D["x"], D["W_r"], None, D["experts"], None, shape, y, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_error(ws) == moe.MOE_ERR_DEVICE_DATA
+
+
 def test_one_hot_and_zero_experts():
     cfg = synth.LayerConfig("onehot", 256, 128, 8, 1, 6, 0.05, None, True)
     L = synth.layer(cfg, 9)
