@@ -77,6 +77,7 @@ constexpr int kXRow = kAtomVals * 2;     // one f16 operand row of an atom
 constexpr unsigned long long kLWaitNs = 2000000000ull;
 constexpr int kPfxMax = kLanePfxMax;     // per-expert table entries (virtual experts + 1)
 constexpr int kEntMax = 512;             // bucket entries staged in shared memory
+constexpr int kOwnMax = 32;              // contributors listed per owned split block
 // f16 range: larger magnitudes round to infinity
 constexpr float kF16Limit = 65520.f;
 
@@ -110,7 +111,8 @@ struct LaneCfg {
   static constexpr int NSCE = 3;                                // scale entries per warp
   static constexpr int WARP_BYTES = D * SLOT + NSCE * SCE;
   static constexpr int SLOTS = NW * D;
-  static constexpr int HEAD = SLOTS * 8 + 5 * kPfxMax * 4 + 2 * NW * 4 + kEntMax * 4;
+  static constexpr int HEAD =
+      SLOTS * 8 + 5 * kPfxMax * 4 + 2 * NW * 4 + kEntMax * 4 + NW * kOwnMax * 4;
   static constexpr int SMEM = 1024 + HEAD + NW * WARP_BYTES;
   static_assert(SLOT % 512 == 0 && SCE % 512 == 0, "64-byte swizzle boxes start on 512 bytes");
   static_assert(NW <= kLaneWarps, "split-block slots are sized for kLaneWarps warps");
@@ -370,8 +372,9 @@ struct LaneWarp {
   int cslot;                // jc % D
   uint32_t cpar;            // (jc / D) & 1
   // the other contributors of the split row block this warp owns at the end
-  // of its range (their warp indices, in atom order); on = -1: none listed
-  int osid[4];
+  // of its range (their warp indices, in atom order, in shared memory); on =
+  // -1: not listed (none, or more than kOwnMax)
+  int* osid;
   int on;
 
   // Per-segment state of the stage loads (nxt entered a new segment).
@@ -824,24 +827,26 @@ __device__ bool run_pass(LaneWarp<PHASE>& W, LaneIt& cur, const FragOfs& f) {
   }
   if (!__shfl_sync(kFull, ok, 0)) return false;
   if (W.on >= 0) {
-    // the contributors listed at setup: their slots in flight together
-    float val[4][NV];
+    // the contributors listed at set-up: four slots in flight at a time
+    for (int q0 = 0; q0 < W.on; q0 += 4) {
+      float val[4][NV];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const bool use = q < W.on;
-      const float* sp = l.part + size_t(use ? W.osid[q] : 0) * SLOTF;
+      for (int q = 0; q < 4; ++q) {
+        const bool use = q0 + q < W.on;
+        const float* sp = l.part + size_t(use ? W.osid[q0 + q] : 0) * SLOTF;
 #pragma unroll
-      for (int n = 0; n < NV; ++n) {
-        int t, row, p;
-        val_pos<PHASE>(n, g, c, t, row, p);
-        val[q][n] = (use && t < R) ? __ldcg(sp + (t * NPROJ + p) * 32 + row) : 0.f;
+        for (int n = 0; n < NV; ++n) {
+          int t, row, p;
+          val_pos<PHASE>(n, g, c, t, row, p);
+          val[q][n] = (use && t < R) ? __ldcg(sp + (t * NPROJ + p) * 32 + row) : 0.f;
+        }
       }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (q0 + q < W.on)
+#pragma unroll
+          for (int n = 0; n < NV; ++n) o.v[n] += val[q][n];
     }
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (q < W.on)
-#pragma unroll
-        for (int n = 0; n < NV; ++n) o.v[n] += val[q][n];
   } else {
     // the contributors are the next non-empty warps of the grid, in atom order
     const int B1 = B0 + l.NA;
@@ -917,6 +922,7 @@ __global__ void __launch_bounds__(LaneCfg<PHASE == 0 ? 2 : 1>::THREADS, 1)
   int* s_off = s_plan + kPfxMax;                                  // [kPfxMax]
   int* s_wsum = s_off + kPfxMax;                                  // [kLW][2]
   int* s_ent = s_wsum + 2 * kLW;                                  // [kEntMax]
+  int* s_own = s_ent + kEntMax;                                   // [kLW][kOwnMax]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
 
@@ -1066,21 +1072,32 @@ __global__ void __launch_bounds__(LaneCfg<PHASE == 0 ? 2 : 1>::THREADS, 1)
   // epilogue once without tokens (no stores), so that its instructions are
   // cached when the phase ends rather than fetched by every warp at once.
   W.on = -1;
+  W.osid = s_own + warp * kOwnMax;
   {
     const int lb0 = (W.A1 - 1) / l.NA * l.NA;  // first atom of the last row block
     if (lb0 >= W.A0 && W.A1 - lb0 < l.NA) {
-      int n = 0, w = W.gw + 1, at = W.A1;
-      while (at < lb0 + l.NA && n < 4) {
-        int nx = W.part.atom_at(w + 1);
-        while (nx == at) {  // warps with empty ranges hold nothing
-          ++w;
-          nx = W.part.atom_at(w + 1);
-        }
-        W.osid[n++] = w;
-        ++w;
-        at = nx;
+      // lanes look up the next warps' first atoms in parallel; the
+      // contributors are the non-empty ones among them, in order
+      const int B1 = lb0 + l.NA;
+      int n = 0, w = W.gw + 1;
+      int at = W.A1;  // first atom of warp w
+      bool done = false;
+      while (!done && n < kOwnMax) {
+        const int nx = W.part.atom_at(w + 1 + lane);  // first atom of warp w + 1 + lane
+        const int cur_at = __shfl_up_sync(kFull, nx, 1);
+        const int my_at = lane == 0 ? at : cur_at;    // first atom of warp w + lane
+        const bool member = my_at < B1 && nx > my_at;  // non-empty and inside the block
+        const unsigned mm = __ballot_sync(kFull, member);
+        const int slot = n + __popc(mm & ((1u << lane) - 1u));
+        if (member && slot < kOwnMax) W.osid[slot] = w + lane;
+        n += __popc(mm);
+        const unsigned past = __ballot_sync(kFull, nx >= B1);
+        done = past != 0;
+        at = __shfl_sync(kFull, nx, 31);
+        w += 32;
       }
-      if (at >= lb0 + l.NA) W.on = n;
+      __syncwarp();
+      if (done && n <= kOwnMax) W.on = n;
     }
   }
   {
