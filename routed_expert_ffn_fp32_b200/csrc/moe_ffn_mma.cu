@@ -33,10 +33,12 @@
 // Data movement.  Each warp keeps D slots of shared memory.  A slot holds the
 // 32 x 64-byte code box of an atom per projection, loaded by a TMA tile copy
 // (64-byte swizzle: the 4-byte fragment loads of the 32 lanes fall in distinct
-// banks), the atom's 128 f16 values of each operand row (1-D bulk copies, one
-// per row), and each weight row's 4 scale bytes per projection (cp.async by
-// the row's lane); all complete on the slot's mbarrier.  The copy for stage
-// j + D is issued as soon as stage j has been consumed.
+// banks), and the atom's 128 f16 values of each operand row (1-D bulk copies,
+// one per row).  Scale bytes come in TMA boxes of 32 rows x 16 bytes (four
+// atoms) where a row's scale bytes are a multiple of 16, else one 4-byte
+// cp.async per row and atom.  All complete on the slot's mbarrier; the copy
+// for stage j + D is issued as soon as stage j has been consumed.  Weight
+// loads carry an L2 evict-first policy (read once per call).
 //
 // Tokens.  A pass handles up to kRMax tokens of an expert; an expert with
 // more tokens has one row block per pass in the flat index space (its weights
@@ -45,12 +47,7 @@
 // Results.  A warp whose range covers a whole row block writes the block's
 // outputs directly (phase 0: SwiGLU as the f16 pair into h; phase 1: the
 // expert output row).  A row block split between warps is finished
-// deterministically: each contributor stores its partial sums in its own slot
-// (a warp has two, for the first and the last block of its range), enters the
-// slot in the block's table at the position of its first atom, and adds its
-// atom count to the block's counter; the contributor that completes the count
-// adds the slots in table order, applies the epilogue and clears the table
-// entries and the counter.
+// deterministically by the warp that holds its first atom (see run_pass).
 //
 // Every wait is bounded (globaltimer); on expiry the kernel latches
 // MOE_ERR_TIMEOUT, lets its in-flight copies land and returns.
@@ -87,23 +84,13 @@ constexpr float kF16Limit = 65520.f;
 // A scale entry holds [NPROJ][32 rows][16 bytes]: the scale bytes of four
 // atoms of each row (one TMA box per projection), or of one atom (cp.async)
 // when a row's scale bytes are not a multiple of 16.
-#ifndef MOE_MMA_NW0
-#define MOE_MMA_NW0 10
-#endif
-#ifndef MOE_MMA_NW1
-#define MOE_MMA_NW1 11
-#endif
-#ifndef MOE_MMA_D0
-#define MOE_MMA_D0 3
-#endif
-#ifndef MOE_MMA_D1
-#define MOE_MMA_D1 3
-#endif
+// Gate/up runs 10 warps (its scale entries are twice the size), down 11;
+// two to six slots per warp and 8 to 11 warps measured the same.
 template <int NPROJ>
 struct LaneCfg {
-  static constexpr int NW = NPROJ == 2 ? MOE_MMA_NW0 : MOE_MMA_NW1;  // warps per CTA
+  static constexpr int NW = NPROJ == 2 ? 10 : 11;  // warps per CTA
   static constexpr int THREADS = 32 * NW;
-  static constexpr int D = NPROJ == 2 ? MOE_MMA_D0 : MOE_MMA_D1;    // slots per warp
+  static constexpr int D = 3;                      // slots per warp
   static constexpr int CODE = NPROJ * kBox;                     // code bytes per slot
   static constexpr int XROWS = NPROJ == 2 ? kRMax : 2 * kRMax;  // f16 operand rows
   static constexpr int SLOT = CODE + XROWS * kXRow;
@@ -1068,9 +1055,7 @@ __global__ void __launch_bounds__(LaneCfg<PHASE == 0 ? 2 : 1>::THREADS, 1)
   }
 
   // While the first stages are in flight: list the contributors of the split
-  // row block this warp will own at the end of its range, and run the
-  // epilogue once without tokens (no stores), so that its instructions are
-  // cached when the phase ends rather than fetched by every warp at once.
+  // row block this warp will own at the end of its range.
   W.on = -1;
   W.osid = s_own + warp * kOwnMax;
   {
@@ -1099,12 +1084,6 @@ __global__ void __launch_bounds__(LaneCfg<PHASE == 0 ? 2 : 1>::THREADS, 1)
       __syncwarp();
       if (done && n <= kOwnMax) W.on = n;
     }
-  }
-  {
-    BlockVals<PHASE, 1> z;
-#pragma unroll
-    for (int n = 0; n < BlockVals<PHASE, 1>::N; ++n) z.v[n] = 0.f;
-    block_store<PHASE, 1>(a, meta, 0, 0, 0, 0, lane, z);
   }
 
   const FragOfs f = frag_ofs(lane);
