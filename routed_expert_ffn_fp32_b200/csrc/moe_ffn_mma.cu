@@ -25,8 +25,9 @@
 // permutation of the block that B follows as well (one 16-byte load of a
 // token row per block and thread).  The two MMAs of a block start from zero
 // and the block's E8M0 scale (2^(s-127), per weight row) multiplies their sum
-// into the float32 accumulators: the result is the same sum of exact products
-// as a scalar loop, accumulated in float32.  Gate/up take the f16 token rows;
+// into the float32 accumulators: every product is exact (f16 x f16 fits a
+// float32) and the sums are float32, though the order of the additions inside
+// an MMA is the hardware's, not a scalar loop's.  Gate/up take the f16 token rows;
 // down takes h as a pair of f16 rows hi + lo (h to 22 significant bits), the
 // two columns of a token summed at the end.
 //
