@@ -251,6 +251,7 @@ def run_ours(args, rank, world, local_rank):
     sampler.stop()
     ms_local = e0.elapsed_time(e1) / args.steps
     ms = max_over_ranks(ms_local, dist, dev)
+    step_pctl = step_percentiles(graphs, ncyc, stream, args.steps)
     assert moe.moe_get_error(ws, stream) == 0
     value = weak_scaling_value(T, world, ms)
 
@@ -366,6 +367,7 @@ def run_ours(args, rank, world, local_rank):
         "layer_hbm_gbs": round(layer_gbs, 1),
         "activated_bytes_per_call": int(bytes_per_call),
         "roofline": roofline, "clocks": clocks, "e2e": e2e,
+        "step_ms_pctl": step_pctl,
         "gpu_launches": launches_per_step * args.steps,
     }
     extra = {}
@@ -519,6 +521,29 @@ def run_sweep(args, local_rank):
                        "weights_gb": round(NL * (cfg.E + 1) * expert_bytes(cfg) / 1e9, 2)},
             "hbm_peak_gbs": peaks["hbm_gbs"], "sweep": rows,
             "crossover_T_gemm_over_gemv_mxfp4": cross}
+
+
+def step_percentiles(graphs, ncyc, stream, steps, n=200):
+    """p10 / median / p90 of single-step times (ms) from a separate pass of n
+    replays, one event pair per step (after the timed region, so the headline
+    timing carries no per-step events).  None if anything goes wrong."""
+    try:
+        import torch
+        n = min(n, steps)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n)]
+        with torch.cuda.stream(stream):
+            for i in range(n):
+                ev[i][0].record(stream)
+                graphs[i % ncyc].replay()
+                ev[i][1].record(stream)
+            stream.synchronize()
+        t = np.array([a.elapsed_time(b) for a, b in ev])
+        return {"p10": round(float(np.percentile(t, 10)), 5),
+                "median": round(float(np.median(t)), 5),
+                "p90": round(float(np.percentile(t, 90)), 5), "steps": n}
+    except Exception:
+        return None
 
 
 def measured_traffic(bytes_per_launch: float):
