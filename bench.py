@@ -6,11 +6,16 @@ FFNs, combine) on one batch of T tokens.  Weights are kept cold in L2 by
 cycling over NL independent copies of the layer (inputs larger than L2).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--T T]
+                    [--workload NAME] [--T T] [--sweep]
 
-Prints one JSON line (rank 0).  With N > 1 (torchrun) every rank runs its own
-batches (independent decode streams, no collective on the data path): weak
-scaling, value = tokens of all ranks / max-over-ranks time.
+Prints one JSON line (rank 0).  The headline is the decode/verify layer
+(H 4096, I 1408, 64 experts, top-2, T = 5); the line's "extra" object holds
+every other workload of the benchmark with its own roofline: the same layer at
+T = 1, the fine-grained layer (256 experts, top-8, shared expert) at T = 1 and
+5, the prefill chunk at T = 2048 and 4096 on the tensor-core path, and the
+crossover of the multi-layer batch sweep.  With N > 1 (torchrun) every rank
+runs its own batches (independent decode streams, no collective on the data
+path): weak scaling, value = tokens of all ranks / max-over-ranks time.
 """
 from __future__ import annotations
 
@@ -30,9 +35,10 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE layer tokens/s; decode HBM GB/s and prefill FP4 TFLOPS as % of roofline"
 DEFAULT_WORKLOAD = "decode_h4096_i1408_e64_k2"
 DEFAULT_T = 5
+FIELDS = ("gate_q", "gate_s", "up_q", "up_s", "down_q", "down_s")
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
@@ -46,10 +52,12 @@ def parse():
     ap.add_argument("--path", choices=["auto", "gemv", "gemm"], default="auto")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--extra-steps", type=int, default=200,
+                    help="timed steps of each extra workload (prefill: a quarter)")
     ap.add_argument("--sweep", action="store_true",
-                    help="the multi-layer cold-cache batch sweep: GEMV and GEMM paths per T, "
-                         "and the crossover (prints its own JSON line)")
-    a = ap.parse_args()
+                    help="the multi-layer cold-cache batch sweep with more repetitions "
+                         "(prints its own JSON line)")
+    a = ap.parse_args(argv)
     a.warmup = max(3, a.warmup)
     return a
 
@@ -141,386 +149,218 @@ def weak_scaling_value(tokens_per_rank: int, world: int, ms: float) -> float:
 # ------------------------------------------------------------- workload ----
 def workload(name: str, T: int):
     from routed_expert_ffn_fp32_b200 import synth
-    cfg = synth.CONFIGS[name]
-    return cfg.with_T(T)
+    return synth.CONFIGS[name].with_T(T)
+
+
+def expert_bytes(cfg) -> int:
+    """Algorithmic bytes of one MXFP4 expert: codes + scales of its three matrices."""
+    return 3 * (cfg.H * cfg.I // 2 + cfg.H * cfg.I // 32)
 
 
 def activated_bytes(cfg, counts: np.ndarray) -> int:
     """Algorithmic bytes of one call: codes + scales of every activated expert."""
-    per = 3 * (cfg.H * cfg.I // 2 + cfg.H * cfg.I // 32)
-    n = int((counts > 0).sum()) + (1 if cfg.shared else 0)
-    return n * per
+    n = int((np.asarray(counts) > 0).sum()) + (1 if cfg.shared else 0)
+    return n * expert_bytes(cfg)
 
 
-def expert_bytes(cfg) -> int:
-    return 3 * (cfg.H * cfg.I // 2 + cfg.H * cfg.I // 32)
+def ffn_flops(cfg, T: int) -> float:
+    """FLOPs of the expert FFNs of one call: 3 projections x 2 H I per row."""
+    return 6.0 * cfg.H * cfg.I * T * (cfg.k + (1 if cfg.shared else 0))
 
 
-# ------------------------------------------------------------ our arm ------
-def run_ours(args, rank, world, local_rank):
+def workload_config(cfg, T, prec_name, path_name, NL) -> dict:
+    return {"workload": cfg.name, "T": T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
+            "shared": cfg.shared, "weights": "MXFP4 (E2M1 + E8M0 per 32)",
+            "activations": "bf16" if prec_name == "exact" else "MXFP4 (quantised)",
+            "accumulate": "f32", "path": path_name, "layer_copies": NL,
+            "l2": f"inputs larger than L2: {NL} layer copies "
+                  f"({NL * (cfg.E + cfg.shared) * expert_bytes(cfg) / 1e9:.2f} GB) cycled"}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "source": "measured (MEASURED_PEAKS.json: STREAM-style copy, cuBLAS bf16 burst)"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def measured_traffic(record: str, bytes_per_launch: float):
+    """DRAM bytes per FFN call from a committed ncu record (profiles/<record>),
+    scaled by the activated bytes of this workload (traffic grows with them);
+    None once the kernel source differs from the one the counters were taken
+    on, or when there is no record."""
+    import hashlib
+    rec = os.path.join(ROOT, "profiles", record)
+    if not os.path.exists(rec):
+        return None
+    d = json.load(open(rec))
+    src = os.path.join(ROOT, d["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != d["source_sha256"]:
+        return None
+    return int(d["dram_bytes_per_call"] / d["algorithmic_bytes_per_call"] * bytes_per_launch)
+
+
+# ---------------------------------------------------------- device layers ---
+class LayerSet:
+    """NL independent device copies of one layer's expert weights (every call
+    of a cycle reads cold weights) and any number of routers over them."""
+
+    def __init__(self, cfg, NL, dev, seed=0):
+        import torch  # noqa: F401
+        from routed_expert_ffn_fp32_b200 import moe, synth
+        self.cfg = cfg
+        L = synth.layer(cfg, seed=seed, T=1)
+        ex0 = moe.Experts.from_numpy(L["experts"], dev)
+        sh0 = moe.Experts.from_numpy(L["shared"], dev) if cfg.shared else None
+        self.layers = [(ex0, sh0)]
+        for _ in range(NL - 1):
+            ex = moe.Experts(**{f: getattr(ex0, f).clone() for f in FIELDS})
+            sh = None if sh0 is None else moe.Experts(**{f: getattr(sh0, f).clone() for f in FIELDS})
+            self.layers.append((ex, sh))
+        self.host = L      # host copy (router, first layer's weights) for the oracle baseline
+        self.dev = dev
+
+    def router(self, rcfg, seed=0):
+        import torch
+        from routed_expert_ffn_fp32_b200 import synth
+        W_r, bias = synth.router(rcfg, seed)
+        return (torch.from_numpy(W_r).to(self.dev),
+                None if bias is None else torch.from_numpy(bias).to(self.dev))
+
+
+def measure(ls, router, rcfg, T, path, prec, steps, warmup, stream, NX=8, seed0=0,
+            ffn=True, sampler=None, dist=None):
+    """Time NL-cycled whole-layer calls (CUDA graphs, one per layer copy and
+    batch) and, with ffn, the expert-FFN call alone on the same routed batches.
+    Returns timings (ms per call), realised activated bytes and the graphs."""
     import torch
-    from routed_expert_ffn_fp32_b200 import build, moe, synth
-
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    build.build()
-    moe.load_library()
-    cfg = workload(args.workload, args.T)
-    T, NL = cfg.T, args.layers
-    PREC, PATH = _consts(args)
-    L = synth.layer(cfg, seed=0)
-    W_r, bias = L["W_r"], L["bias"]
-    ex0 = moe.Experts.from_numpy(L["experts"], dev)
-    sh0 = moe.Experts.from_numpy(L["shared"], dev) if cfg.shared else None
-    layers = [(ex0, sh0)]
-    for _ in range(NL - 1):   # independent copies: every call reads cold weights
-        ex = moe.Experts(**{f: getattr(ex0, f).clone() for f in
-                            ("gate_q", "gate_s", "up_q", "up_s", "down_q", "down_s")})
-        sh = None if sh0 is None else moe.Experts(**{f: getattr(sh0, f).clone() for f in
-                                                     ("gate_q", "gate_s", "up_q", "up_s",
-                                                      "down_q", "down_s")})
-        layers.append((ex, sh))
-    Wd = torch.from_numpy(W_r).to(dev)
-    bd = None if bias is None else torch.from_numpy(bias).to(dev)
-    NX = 16
-    xs_np = [synth.activations(cfg, seed=1000 * rank + i, T=T) for i in range(NX)]
+    from routed_expert_ffn_fp32_b200 import moe, synth
+    dev = ls.dev
+    cfg = rcfg.with_T(T)
+    Wd, bd = router
+    NL = len(ls.layers)
+    xs_np = [synth.activations(cfg, seed=seed0 + i, T=T) for i in range(NX)]
     xs = [torch.from_numpy(a.view(np.int16)).to(dev) for a in xs_np]
     shape = moe.shape_of(T, cfg.H, cfg.I, cfg.E, cfg.k)
-    stream = torch.cuda.Stream(dev)
-    ws = moe.make_workspace(shape, PATH, PREC, cfg.shared, dev, stream)
+    ws = moe.make_workspace(shape, path, prec, cfg.shared, dev, stream)
     y = torch.empty((T, cfg.H), dtype=torch.int16, device=dev)
     idx = torch.empty((T, cfg.k), dtype=torch.int32, device=dev)
     wts = torch.empty((T, cfg.k), dtype=torch.float32, device=dev)
+    ncyc = int(np.lcm(NL, NX))
 
     def call(i, st):
-        ex, sh = layers[i % NL]
-        moe.moe_layer_forward(xs[i % NX], Wd, bd, ex, sh, shape, y, ws, PATH, PREC, idx, wts,
+        ex, sh = ls.layers[i % NL]
+        moe.moe_layer_forward(xs[i % NX], Wd, bd, ex, sh, shape, y, ws, path, prec, idx, wts,
                               stream=st)
 
-    # one graph per (layer copy, batch) pair in the cycle
-    ncyc = int(np.lcm(NL, NX))
+    nbytes = []
     with torch.cuda.stream(stream):
-        for i in range(min(ncyc, 4)):
+        for i in range(NX):
             call(i, stream)
-        stream.synchronize()
+            stream.synchronize()
+            nbytes.append(activated_bytes(cfg, np.bincount(idx.cpu().numpy().reshape(-1),
+                                                           minlength=cfg.E)))
         graphs = []
         for i in range(ncyc):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 call(i, stream)
             graphs.append(g)
-    assert moe.moe_get_error(ws, stream) == 0
-
-    # routed activated bytes per call (the bench reports the realised mean)
-    act_bytes = []
-    with torch.cuda.stream(stream):
-        for i in range(NX):
-            call(i, stream)
-            stream.synchronize()
-            counts = np.bincount(idx.cpu().numpy().reshape(-1), minlength=cfg.E)
-            act_bytes.append(activated_bytes(cfg, counts))
-    bytes_per_call = float(np.mean(act_bytes))
-
-    dist = None
-    if world > 1:
-        import torch.distributed as dist  # noqa: F811
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    sampler = ClockSampler(local_rank)
-    sampler.start()
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
+        for i in range(warmup):
             graphs[i % ncyc].replay()
         stream.synchronize()
-        barrier()
+        if dist is not None:
+            dist.barrier()
         torch.cuda.synchronize(dev)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         h0 = time.perf_counter()
+        if sampler is not None:
+            sampler.start()
         e0.record(stream)
-        for i in range(args.steps):
+        for i in range(steps):
             graphs[i % ncyc].replay()
         e1.record(stream)
         stream.synchronize()
         h1 = time.perf_counter()
+        if sampler is not None:
+            sampler.stop()
         torch.cuda.synchronize(dev)
-        barrier()
-    sampler.stop()
-    ms_local = e0.elapsed_time(e1) / args.steps
-    ms = max_over_ranks(ms_local, dist, dev)
-    step_pctl = step_percentiles(graphs, ncyc, stream, args.steps)
-    assert moe.moe_get_error(ws, stream) == 0
-    value = weak_scaling_value(T, world, ms)
-
-    # ---- dominant kernels: expert FFN (gate/up + down) timed alone -------------
+        if dist is not None:
+            dist.barrier()
+    st = moe.moe_get_error(ws, stream)
+    assert st == 0, f"device status {st}"
+    out = {"ms_layer": e0.elapsed_time(e1) / steps, "bytes_layer": float(np.mean(nbytes)),
+           "graphs": graphs, "ncyc": ncyc, "h0": h0, "h1": h1, "xs_np": xs_np, "xs": xs,
+           "ws": ws, "shape": shape, "y": y}
+    if not ffn:
+        return out
+    # the expert-FFN call alone (plan, scaled f16 token rows or the MXFP4
+    # gather, gate/up + SwiGLU, down) over the same routed batches
     offs = torch.empty(cfg.E + 1, dtype=torch.int32, device=dev)
     cnts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
     ents = torch.empty(T * cfg.k, dtype=torch.int32, device=dev)
     rows = T * cfg.k + (T if cfg.shared else 0)
     partial = torch.empty((rows, cfg.H), dtype=torch.float32, device=dev)
-    ffn_graphs, ffn_bytes = [], []
+    fgraphs, fbytes, keep = [], [], []
     with torch.cuda.stream(stream):
         for i in range(ncyc):
-            ex, sh = layers[i % NL]
+            ex, sh = ls.layers[i % NL]
             moe.moe_route_topk(xs[i % NX], Wd, bd, shape, idx, wts, ws, stream=stream)
             moe.moe_bucket(idx, shape, cnts, offs, ents, ws, stream=stream)
             stream.synchronize()
-            counts = cnts.cpu().numpy()
-            ffn_bytes.append(activated_bytes(cfg, counts))
-            # each graph keeps its own routing in its own buffers
-            o_i, e_i = offs.clone(), ents.clone()
+            fbytes.append(activated_bytes(cfg, cnts.cpu().numpy()))
+            o_i, e_i = offs.clone(), ents.clone()   # each graph keeps its own routing
+            keep.append((o_i, e_i))
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                moe.moe_expert_ffn_mxfp4(ex, sh, xs[i % NX], o_i, e_i, shape, partial, ws,
-                                         PATH, PREC, stream=stream)
-            ffn_graphs.append((g, o_i, e_i))
-        for i in range(args.warmup):
-            ffn_graphs[i % ncyc][0].replay()
+                moe.moe_expert_ffn_mxfp4(ex, sh, xs[i % NX], o_i, e_i, shape, partial, ws, path,
+                                         prec, stream=stream)
+            fgraphs.append(g)
+        for i in range(warmup):
+            fgraphs[i % ncyc].replay()
         stream.synchronize()
         f0 = torch.cuda.Event(enable_timing=True)
         f1 = torch.cuda.Event(enable_timing=True)
-        nrep = max(args.steps, ncyc)
+        nrep = max(steps, ncyc)
         f0.record(stream)
         for i in range(nrep):
-            ffn_graphs[i % ncyc][0].replay()
+            fgraphs[i % ncyc].replay()
         f1.record(stream)
         stream.synchronize()
-    ffn_ms = f0.elapsed_time(f1) / nrep
-    ffn_b = float(np.mean([ffn_bytes[i % ncyc] for i in range(nrep)]))
-    peaks = load_peaks()
-    achieved = ffn_b / (ffn_ms / 1e3) / 1e9
-    flops = 6.0 * cfg.H * cfg.I * T * (cfg.k + (1 if cfg.shared else 0))
-    tflops = flops / (ffn_ms / 1e3) / 1e12
-    # AUTO takes the tensor-core kernels for MXFP4 activations at every batch size
-    uses_tc = PREC == moe.MOE_ACT_MXFP4 and PATH in (moe.MOE_PATH_GEMM, moe.MOE_PATH_AUTO)
-    fp4_peak = peaks["bf16_tflops"] * 4.0  # dense FP4 = 4 x dense bf16 (nominal ratio)
-    t_hbm = ffn_b / (peaks["hbm_gbs"] * 1e9)
-    t_tc = flops / (fp4_peak * 1e12)
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": None, "kernel": "expert FFN call (plan, f16 token rows, gate/up + SwiGLU, down)",
-                "peak_source": peaks["source"], "bytes_per_launch": int(ffn_b),
-                "launch_ms": round(ffn_ms, 5)}
-    if not uses_tc and cfg.T <= 512:
-        roofline["traffic"] = measured_traffic(ffn_b)
-        roofline["traffic_source"] = "ncu dram__bytes_read.sum + dram__bytes_write.sum of k_ffn_mma " \
-                                     "(profiles/k_ffn_mma_decode64_t5.json), scaled by activated bytes"
+    assert moe.moe_get_error(ws, stream) == 0
+    out["ms_ffn"] = f0.elapsed_time(f1) / nrep
+    out["bytes_ffn"] = float(np.mean([fbytes[i % ncyc] for i in range(nrep)]))
+    return out
+
+
+def roofline_of(cfg, T, r, peaks, uses_tc, record=None) -> dict:
+    """Roofline of the expert-FFN call: algorithmic bytes (activated experts) /
+    its measured time against the measured HBM copy peak; on the tensor-core
+    path also FP4 TFLOP/s against the FP4 peak and the attainable fraction."""
+    ms, b = r["ms_ffn"], r["bytes_ffn"]
+    achieved = b / (ms / 1e3) / 1e9
+    out = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+           "frac": round(achieved / peaks["hbm_gbs"], 4),
+           "traffic": measured_traffic(record, b) if record else None,
+           "kernel": "expert FFN call (plan, scaled f16 token rows, gate/up + SwiGLU, down)",
+           "peak_source": peaks["source"], "bytes_per_launch": int(b), "launch_ms": round(ms, 5)}
     if uses_tc:
-        roofline["kernel"] = "expert FFN on tcgen05 kind::mxf4 (gate/up + SwiGLU + requant, down)"
-        roofline["tensor"] = {
-            "achieved_tflops": round(tflops, 1), "fp4_peak_tflops": round(fp4_peak, 1),
-            "frac_of_fp4_peak": round(tflops / fp4_peak, 4),
-            "fp4_peak_source": "measured bf16 burst x 4 (nominal dense FP4/bf16 ratio)",
-            "flops_per_launch": flops,
-            "attainable_frac": round(max(t_hbm, t_tc) / (ffn_ms / 1e3), 4),
-            "bound_by": "hbm" if t_hbm >= t_tc else "tensor"}
-    layer_gbs = bytes_per_call / (ms_local / 1e3) / 1e9
-
-    # ---- end to end through the C ABI with host buffers ------------------------
-    xh = [torch.from_numpy(a.view(np.int16)).pin_memory() for a in xs_np]
-    yh = torch.empty((T, cfg.H), dtype=torch.int16).pin_memory()
-    xd = torch.empty_like(xs[0])
-    n_e2e = min(args.steps, 2000)
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            xd.copy_(xh[i % NX], non_blocking=True)
-            ex, sh = layers[i % NL]
-            moe.moe_layer_forward(xd, Wd, bd, ex, sh, shape, y, ws, PATH, PREC, stream=stream)
-            yh.copy_(y, non_blocking=True)
-        stream.synchronize()
-        g0 = torch.cuda.Event(enable_timing=True)
-        g1 = torch.cuda.Event(enable_timing=True)
-        g0.record(stream)
-        for i in range(n_e2e):
-            xd.copy_(xh[i % NX], non_blocking=True)
-            ex, sh = layers[i % NL]
-            moe.moe_layer_forward(xd, Wd, bd, ex, sh, shape, y, ws, PATH, PREC, stream=stream)
-            yh.copy_(y, non_blocking=True)
-        g1.record(stream)
-        stream.synchronize()
-    e2e_ms = g0.elapsed_time(g1) / n_e2e
-    e2e = {"value": round(T / (e2e_ms / 1e3), 1), "unit": "tokens/s",
-           "h2d_bytes_per_step": T * cfg.H * 2, "d2h_bytes_per_step": T * cfg.H * 2,
-           "ms_per_step": round(e2e_ms, 5), "api": "moe_layer_forward (eager, ctypes)"}
-
-    # route (fused for T <= 32) + gate/up + down + combine; the tensor-core path
-    # adds the activation gather and the work-item plan
-    launches_per_step = (4 if T <= 32 else 6) + (2 if uses_tc else 0)
-    clocks = sampler.summary(h0, h1)
-    out = {
-        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32" if PREC == moe.MOE_ACT_EXACT else "mxfp4 x mxfp4 -> f32",
-        "data": "synthetic",
-        "config": {"workload": cfg.name, "T": T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
-                   "shared": cfg.shared, "weights": "MXFP4 (E2M1 + E8M0 per 32)",
-                   "activations": "bf16" if PREC == moe.MOE_ACT_EXACT else "MXFP4 (quantised)",
-                   "accumulate": "f32", "path": args.path,
-                   "layer_copies": NL,
-                   "l2": f"inputs larger than L2: {NL} layer copies "
-                         f"({NL * cfg.E * expert_bytes(cfg) / 1e9:.2f} GB) cycled",
-                   "parallelism": f"independent streams x{world}"},
-        "layer_hbm_gbs": round(layer_gbs, 1),
-        "activated_bytes_per_call": int(bytes_per_call),
-        "roofline": roofline, "clocks": clocks, "e2e": e2e,
-        "step_ms_pctl": step_pctl,
-        "gpu_launches": launches_per_step * args.steps,
-    }
-    extra = {}
-    if not args.no_extra and args.workload == DEFAULT_WORKLOAD and rank == 0:
-        extra = run_extra(cfg, layers, Wd, bd, stream, dev, args)
-    if extra:
-        out["extra"] = extra
-    ctx = {"L": L, "cfg": cfg, "xs_np": xs_np}
-    return out, ctx
-
-
-def run_extra(cfg, layers, Wd, bd, stream, dev, args):
-    """The same layer at the other batch size of the decode/verify workload."""
-    import torch
-    from routed_expert_ffn_fp32_b200 import moe, synth
-    res = {}
-    for T in (1,) if cfg.T != 1 else (5,):
-        shape = moe.shape_of(T, cfg.H, cfg.I, cfg.E, cfg.k)
-        ws = moe.make_workspace(shape, moe.MOE_PATH_AUTO, moe.MOE_ACT_EXACT, cfg.shared, dev,
-                                stream)
-        y = torch.empty((T, cfg.H), dtype=torch.int16, device=dev)
-        idx = torch.empty((T, cfg.k), dtype=torch.int32, device=dev)
-        wts = torch.empty((T, cfg.k), dtype=torch.float32, device=dev)
-        xs = [torch.from_numpy(synth.activations(cfg, 7000 + i, T).view(np.int16)).to(dev)
-              for i in range(8)]
-        NL = len(layers)
-        graphs, nbytes = [], []
-        with torch.cuda.stream(stream):
-            for i in range(NL):
-                ex, sh = layers[i]
-                moe.moe_layer_forward(xs[i % 8], Wd, bd, ex, sh, shape, y, ws,
-                                      moe.MOE_PATH_AUTO, moe.MOE_ACT_EXACT, idx, wts,
-                                      stream=stream)
-                stream.synchronize()
-                nbytes.append(activated_bytes(cfg, np.bincount(idx.cpu().numpy().reshape(-1),
-                                                               minlength=cfg.E)))
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
-                    moe.moe_layer_forward(xs[i % 8], Wd, bd, ex, sh, shape, y, ws,
-                                          moe.MOE_PATH_AUTO, moe.MOE_ACT_EXACT, idx, wts,
-                                          stream=stream)
-                graphs.append(g)
-            for i in range(args.warmup):
-                graphs[i % NL].replay()
-            stream.synchronize()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            n = max(args.steps, 1000)
-            a.record(stream)
-            for i in range(n):
-                graphs[i % NL].replay()
-            b.record(stream)
-            stream.synchronize()
-        ms = a.elapsed_time(b) / n
-        gbs = float(np.mean(nbytes)) / (ms / 1e3) / 1e9
-        res[f"T{T}"] = {"tokens_per_s": round(T / (ms / 1e3), 1), "ms_per_step": round(ms, 5),
-                        "layer_hbm_gbs": round(gbs, 1),
-                        "activated_bytes_per_call": int(np.mean(nbytes))}
-    return res
-
-
-# ----------------------------------------------------- batch-size sweep ----
-def run_sweep(args, local_rank):
-    """Eight independent copies of the fine-grained layer (Zipf 1.2 routing),
-    called in turn so every call reads cold weights; for each batch size the
-    CUDA-core path (exact and MXFP4 activations) and the tensor-core path
-    (MXFP4 activations) are timed as whole layers.  The crossover is the
-    smallest batch at which the tensor-core path beats the CUDA-core path at
-    the same precision."""
-    import torch
-    from routed_expert_ffn_fp32_b200 import build, moe, synth
-
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    build.build()
-    moe.load_library()
-    base = synth.SWEEP
-    NL = synth.SWEEP_LAYERS
-    L = synth.layer(base, seed=0)
-    ex0 = moe.Experts.from_numpy(L["experts"], dev)
-    sh0 = moe.Experts.from_numpy(L["shared"], dev)
-    fields = ("gate_q", "gate_s", "up_q", "up_s", "down_q", "down_s")
-    layers = [(ex0, sh0)] + [
-        (moe.Experts(**{f: getattr(ex0, f).clone() for f in fields}),
-         moe.Experts(**{f: getattr(sh0, f).clone() for f in fields})) for _ in range(NL - 1)]
-    Wd = torch.from_numpy(L["W_r"]).to(dev)
-    bd = torch.from_numpy(L["bias"]).to(dev)
-    stream = torch.cuda.Stream(dev)
-    variants = [("gemv_exact", moe.MOE_PATH_GEMV, moe.MOE_ACT_EXACT),
-                ("gemv_mxfp4", moe.MOE_PATH_GEMV, moe.MOE_ACT_MXFP4),
-                ("gemm_mxfp4", moe.MOE_PATH_GEMM, moe.MOE_ACT_MXFP4)]
-    rows = []
-    for T in synth.SWEEP_T:
-        cfg = base.with_T(T)
-        shape = moe.shape_of(T, cfg.H, cfg.I, cfg.E, cfg.k)
-        NX = 4
-        xs = [torch.from_numpy(synth.activations(cfg, 9000 + i, T).view(np.int16)).to(dev)
-              for i in range(NX)]
-        y = torch.empty((T, cfg.H), dtype=torch.int16, device=dev)
-        idx = torch.empty((T, cfg.k), dtype=torch.int32, device=dev)
-        wts = torch.empty((T, cfg.k), dtype=torch.float32, device=dev)
-        row = {"T": T}
-        nbytes = []
-        for name, path, prec in variants:
-            ws = moe.make_workspace(shape, path, prec, True, dev, stream)
-            ncyc = int(np.lcm(NL, NX))
-            graphs = []
-            with torch.cuda.stream(stream):
-                for i in range(ncyc):
-                    ex, sh = layers[i % NL]
-                    moe.moe_layer_forward(xs[i % NX], Wd, bd, ex, sh, shape, y, ws, path, prec,
-                                          idx, wts, stream=stream)
-                    if name == "gemv_exact":
-                        stream.synchronize()
-                        nbytes.append(activated_bytes(
-                            cfg, np.bincount(idx.cpu().numpy().reshape(-1), minlength=cfg.E)))
-                stream.synchronize()
-                for i in range(ncyc):
-                    ex, sh = layers[i % NL]
-                    g = torch.cuda.CUDAGraph()
-                    with torch.cuda.graph(g, stream=stream):
-                        moe.moe_layer_forward(xs[i % NX], Wd, bd, ex, sh, shape, y, ws, path,
-                                              prec, idx, wts, stream=stream)
-                    graphs.append(g)
-                for i in range(max(args.warmup, 3)):
-                    graphs[i % ncyc].replay()
-                stream.synchronize()
-                n = max(ncyc, min(200, int(2e5 / T)))
-                a = torch.cuda.Event(enable_timing=True)
-                b = torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                for i in range(n):
-                    graphs[i % ncyc].replay()
-                b.record(stream)
-                stream.synchronize()
-            assert moe.moe_get_error(ws, stream) == 0
-            ms = a.elapsed_time(b) / n
-            row[name] = {"tokens_per_s": round(T / (ms / 1e3), 1), "ms_per_step": round(ms, 5)}
-            del graphs, ws
-        act = float(np.mean(nbytes))
-        row["activated_bytes_per_call"] = int(act)
-        for name, _, _ in variants:
-            row[name]["hbm_gbs"] = round(act / (row[name]["ms_per_step"] / 1e3) / 1e9, 1)
-        rows.append(row)
-    cross = next((r["T"] for r in rows
-                  if r["gemm_mxfp4"]["tokens_per_s"] > r["gemv_mxfp4"]["tokens_per_s"]), None)
-    peaks = load_peaks()
-    return {"metric": "MoE layer tokens/s over the batch sweep (cold weights, 8 layers)",
-            "unit": "tokens/s", "n_gpus": 1, "data": "synthetic",
-            "config": {"workload": base.name, "layers": NL, "T": list(synth.SWEEP_T),
-                       "weights_gb": round(NL * (cfg.E + 1) * expert_bytes(cfg) / 1e9, 2)},
-            "hbm_peak_gbs": peaks["hbm_gbs"], "sweep": rows,
-            "crossover_T_gemm_over_gemv_mxfp4": cross}
+        flops = ffn_flops(cfg, T)
+        fp4_peak = peaks["bf16_tflops"] * 4.0  # dense FP4 = 4 x dense bf16 (nominal ratio)
+        t_hbm = b / (peaks["hbm_gbs"] * 1e9)
+        t_tc = flops / (fp4_peak * 1e12)
+        tflops = flops / (ms / 1e3) / 1e12
+        out["kernel"] = "expert FFN on tcgen05 kind::mxf4 (MXFP4 gather, gate/up + SwiGLU + requant, down)"
+        out["tensor"] = {"achieved_tflops": round(tflops, 1), "fp4_peak_tflops": round(fp4_peak, 1),
+                         "frac_of_fp4_peak": round(tflops / fp4_peak, 4),
+                         "fp4_peak_source": "measured bf16 burst x 4 (nominal dense FP4/bf16 ratio)",
+                         "flops_per_launch": flops,
+                         "attainable_frac": round(max(t_hbm, t_tc) / (ms / 1e3), 4),
+                         "bound_by": "hbm" if t_hbm >= t_tc else "tensor"}
+    return out
 
 
 def step_percentiles(graphs, ncyc, stream, steps, n=200):
@@ -546,29 +386,187 @@ def step_percentiles(graphs, ncyc, stream, steps, n=200):
         return None
 
 
-def measured_traffic(bytes_per_launch: float):
-    """DRAM bytes per FFN call from the committed ncu record of the decode GEMV,
-    scaled by the activated bytes of this workload (traffic grows with them);
-    None once the kernel source has changed since the counters were taken, or
-    for another kernel."""
-    import hashlib
-    rec = os.path.join(ROOT, "profiles", "k_ffn_mma_decode64_t5.json")
-    if not os.path.exists(rec):
-        return None
-    d = json.load(open(rec))
-    src = os.path.join(ROOT, d["source"])
-    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != d["source_sha256"]:
-        return None
-    return int(d["dram_bytes_per_call"] / d["algorithmic_bytes_per_call"] * bytes_per_launch)
+def e2e_measure(ls, router, cfg, T, path, prec, r, steps, warmup, stream):
+    """The same metric end to end through the public API: every step copies
+    its batch from pinned host memory, calls moe_layer_forward eagerly and
+    reads the bf16 output back into pinned host memory."""
+    import torch
+    from routed_expert_ffn_fp32_b200 import moe
+    Wd, bd = router
+    NL = len(ls.layers)
+    xh = [torch.from_numpy(a.view(np.int16)).pin_memory() for a in r["xs_np"]]
+    NX = len(xh)
+    yh = torch.empty((T, cfg.H), dtype=torch.int16).pin_memory()
+    xd = torch.empty_like(r["xs"][0])
+    y, ws, shape = r["y"], r["ws"], r["shape"]
+    n = min(steps, 2000)
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            xd.copy_(xh[i % NX], non_blocking=True)
+            ex, sh = ls.layers[i % NL]
+            moe.moe_layer_forward(xd, Wd, bd, ex, sh, shape, y, ws, path, prec, stream=stream)
+            yh.copy_(y, non_blocking=True)
+        stream.synchronize()
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for i in range(n):
+            xd.copy_(xh[i % NX], non_blocking=True)
+            ex, sh = ls.layers[i % NL]
+            moe.moe_layer_forward(xd, Wd, bd, ex, sh, shape, y, ws, path, prec, stream=stream)
+            yh.copy_(y, non_blocking=True)
+        g1.record(stream)
+        stream.synchronize()
+    ms = g0.elapsed_time(g1) / n
+    return {"value": round(T / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": T * cfg.H * 2, "d2h_bytes_per_step": T * cfg.H * 2,
+            "ms_per_step": round(ms, 5), "api": "moe_layer_forward (eager, ctypes)"}
 
 
-def load_peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        d = json.load(open(p))
-        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
-                "source": "measured (MEASURED_PEAKS.json: STREAM-style copy)"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+# ------------------------------------------------------------ our arm ------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from routed_expert_ffn_fp32_b200 import build, moe, synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    build.build()
+    moe.load_library()
+    cfg = workload(args.workload, args.T)
+    T, NL = cfg.T, args.layers
+    PREC, PATH = _consts(args)
+    peaks = load_peaks()
+    stream = torch.cuda.Stream(dev)
+    ls = LayerSet(cfg, NL, dev)
+    router = ls.router(cfg)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist  # noqa: F811
+
+    sampler = ClockSampler(local_rank)
+    r = measure(ls, router, cfg, T, PATH, PREC, args.steps, args.warmup, stream,
+                NX=16, seed0=1000 * rank, sampler=sampler, dist=dist)
+    ms = max_over_ranks(r["ms_layer"], dist, dev)
+    value = weak_scaling_value(T, world, ms)
+    uses_tc = PREC == moe.MOE_ACT_MXFP4 and PATH in (moe.MOE_PATH_GEMM, moe.MOE_PATH_AUTO)
+    record = None if uses_tc else "k_ffn_mma_decode64_t5.json"
+    roof = roofline_of(cfg, T, r, peaks, uses_tc, record)
+    if roof.get("traffic") is not None:
+        roof["traffic_source"] = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of both "
+                                  "k_ffn_mma phases (profiles/k_ffn_mma_decode64_t5.json), "
+                                  "scaled by activated bytes")
+    e2e = e2e_measure(ls, router, cfg, T, PATH, PREC, r, args.steps, args.warmup, stream)
+    # route (fused for T <= 32) + gate/up + down + combine; the tensor-core
+    # path adds the activation gather and the work-item plan
+    launches_per_step = (4 if T <= 32 else 7) + (2 if uses_tc else 0)
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if PREC == moe.MOE_ACT_EXACT else "mxfp4 x mxfp4 -> f32",
+        "data": "synthetic",
+        "config": dict(workload_config(cfg, T, args.precision, args.path, NL),
+                       parallelism=f"independent streams x{world}"),
+        "layer_hbm_gbs": round(r["bytes_layer"] / (r["ms_layer"] / 1e3) / 1e9, 1),
+        "activated_bytes_per_call": int(r["bytes_layer"]),
+        "roofline": roof, "clocks": sampler.summary(r["h0"], r["h1"]), "e2e": e2e,
+        "step_ms_pctl": step_percentiles(r["graphs"], r["ncyc"], stream, args.steps),
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    del r
+    if not args.no_extra and args.workload == DEFAULT_WORKLOAD and rank == 0:
+        out["extra"] = run_extra(ls, router, args, stream, dev, peaks)
+    ctx = {"L": ls.host, "cfg": cfg}
+    return out, ctx
+
+
+def run_extra(ls64, router64, args, stream, dev, peaks):
+    """Every other workload of the benchmark, each with its own roofline."""
+    from routed_expert_ffn_fp32_b200 import moe, synth
+    ex = {}
+    steps = max(10, args.extra_steps)
+    E, G, A, M = moe.MOE_ACT_EXACT, moe.MOE_PATH_GEMV, moe.MOE_PATH_AUTO, moe.MOE_ACT_MXFP4
+
+    def entry(ls, router, rcfg, T, path, prec, n, record=None, uses_tc=False):
+        r = measure(ls, router, rcfg, T, path, prec, n, max(3, min(args.warmup, 20)), stream,
+                    seed0=7000)
+        cfg = rcfg.with_T(T)
+        e = {"tokens_per_s": round(T / (r["ms_layer"] / 1e3), 1),
+             "ms_per_step": round(r["ms_layer"], 5),
+             "layer_hbm_gbs": round(r["bytes_layer"] / (r["ms_layer"] / 1e3) / 1e9, 1),
+             "activated_bytes_per_call": int(r["bytes_layer"]),
+             "roofline": roofline_of(cfg, T, r, peaks, uses_tc, record),
+             "config": workload_config(cfg, T, "mxfp4" if prec == M else "exact",
+                                       "auto" if path == A else "gemv", len(ls.layers))}
+        return e
+
+    ex["decode64_T1"] = entry(ls64, router64, synth.DECODE64, 1, A, E, steps,
+                              record="k_ffn_mma_decode64_t5.json")
+    fg = synth.FINEGRAINED
+    lsf = LayerSet(fg.with_T(1), len(ls64.layers), dev)
+    rf = lsf.router(fg)
+    ex["finegrained_T1"] = entry(lsf, rf, fg, 1, A, E, steps)
+    ex["finegrained_T5"] = entry(lsf, rf, fg, 5, A, E, steps)
+    pre = synth.PREFILL
+    rp = lsf.router(pre)
+    for T in (2048, 4096):
+        ex[f"prefill_T{T}"] = entry(lsf, rp, pre, T, A, M, max(10, steps // 4), uses_tc=True)
+    ex["sweep"] = sweep_rows(lsf, rp, synth.SWEEP, stream, reps=max(10, steps // 10),
+                             variants=("gemv_mxfp4", "gemm_mxfp4"))
+    return ex
+
+
+# ----------------------------------------------------- batch-size sweep ----
+SWEEP_VARIANTS = {"gemv_exact": ("gemv", "exact"), "gemv_mxfp4": ("gemv", "mxfp4"),
+                  "gemm_mxfp4": ("gemm", "mxfp4")}
+
+
+def sweep_rows(ls, router, base, stream, reps, variants):
+    """Eight cold copies of the fine-grained layer, Zipf 1.2 routing: for each
+    batch size of the sweep, whole-layer tokens/s of each path, and the
+    crossover (the smallest batch at which the tensor-core path beats the
+    CUDA-core path at the same MXFP4 activations)."""
+    from routed_expert_ffn_fp32_b200 import moe, synth
+    rows = []
+    for T in synth.SWEEP_T:
+        row = {"T": T}
+        for name in variants:
+            path_n, prec_n = SWEEP_VARIANTS[name]
+            path = moe.MOE_PATH_GEMM if path_n == "gemm" else moe.MOE_PATH_GEMV
+            prec = moe.MOE_ACT_MXFP4 if prec_n == "mxfp4" else moe.MOE_ACT_EXACT
+            r = measure(ls, router, base, T, path, prec, max(len(ls.layers), reps), 3, stream,
+                        NX=4, seed0=9000, ffn=False)
+            row[name] = {"tokens_per_s": round(T / (r["ms_layer"] / 1e3), 1),
+                         "ms_per_step": round(r["ms_layer"], 5),
+                         "hbm_gbs": round(r["bytes_layer"] / (r["ms_layer"] / 1e3) / 1e9, 1)}
+            row["activated_bytes_per_call"] = int(r["bytes_layer"])
+            del r
+        rows.append(row)
+    cross = None
+    if "gemv_mxfp4" in variants and "gemm_mxfp4" in variants:
+        cross = next((r["T"] for r in rows
+                      if r["gemm_mxfp4"]["tokens_per_s"] > r["gemv_mxfp4"]["tokens_per_s"]), None)
+    return {"workload": base.name, "layers": len(ls.layers), "rows": rows,
+            "crossover_T_gemm_over_gemv_mxfp4": cross}
+
+
+def run_sweep(args, local_rank):
+    import torch
+    from routed_expert_ffn_fp32_b200 import build, moe, synth
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    build.build()
+    moe.load_library()
+    base = synth.SWEEP
+    ls = LayerSet(base.with_T(1), synth.SWEEP_LAYERS, dev)
+    stream = torch.cuda.Stream(dev)
+    res = sweep_rows(ls, ls.router(base), base, stream, reps=200,
+                     variants=("gemv_exact", "gemv_mxfp4", "gemm_mxfp4"))
+    peaks = load_peaks()
+    return {"metric": "MoE layer tokens/s over the batch sweep (cold weights, 8 layers)",
+            "unit": "tokens/s", "n_gpus": 1, "data": "synthetic", "hbm_peak_gbs": peaks["hbm_gbs"],
+            "config": {"workload": base.name, "layers": synth.SWEEP_LAYERS,
+                       "T": list(synth.SWEEP_T)}, **res}
 
 
 # ------------------------------------------------------- oracle on the CPU ---
@@ -577,12 +575,10 @@ def oracle_sample(cfg, L, x_bits, budget_s: float):
     import oracle as O
     t0 = time.perf_counter()
     tokens = 0
-    calls = 0
     while True:
         row = x_bits[tokens % x_bits.shape[0]: tokens % x_bits.shape[0] + 1]
         O.layer_forward(row, L["W_r"], L["bias"], L["experts"], L["shared"], cfg.k)
         tokens += 1
-        calls += 1
         if time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
@@ -599,11 +595,14 @@ def blas_threads() -> int:
 
 
 def cpu_baseline(ctx, budget_s=15.0):
+    from routed_expert_ffn_fp32_b200 import synth
     cfg = ctx["cfg"]
-    v, n, dt = oracle_sample(cfg, ctx["L"], ctx["xs_np"][0], budget_s)
-    return {"value": round(v, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} tokens of {cfg.name} (one token per oracle call, fp64 numpy; "
-                      f"{dt:.1f} s)"}
+    x = synth.activations(cfg, seed=0, T=cfg.T)
+    v, n, dt = oracle_sample(cfg, ctx["L"], x, budget_s)
+    return {"value": round(v, 3), "unit": "tokens/s", "cores": blas_threads(),
+            "host_cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{n} tokens of {cfg.name} (one token per oracle call, fp64 numpy on "
+                      f"{blas_threads()} BLAS threads of {os.cpu_count()} host cores; {dt:.1f} s)"}
 
 
 def run_reference(args, rank, world):
@@ -629,10 +628,11 @@ def run_reference(args, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E,
-                       "k": cfg.k, "sample": "one token of the batch per step"},
+            "config": dict(workload_config(cfg, cfg.T, args.precision, args.path, args.layers),
+                           parallelism=f"independent streams x{world}"),
             "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": cores,
-                             "kind": "oracle", "sample": "one token per step, fp64 numpy oracle"},
+                             "host_cores": os.cpu_count(), "kind": "oracle",
+                             "sample": "one token of the batch per step, fp64 numpy oracle"},
             "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 

@@ -57,9 +57,12 @@
  *
  * Workspace: `ws` is caller-owned device memory of at least
  * moe_workspace_bytes(...) bytes, zeroed once by moe_workspace_init() before
- * its first use.  Kernels leave its counters at zero, so one workspace serves
- * any number of calls, including calls replayed from a CUDA graph, as long as
- * calls sharing a workspace are ordered on one stream.
+ * its first use.  Its first 16 bytes hold the latched error (status, detail),
+ * the wait limit and the debug switches (moe_workspace_set_limits); every call
+ * clears the other scratch it relies on itself, so one workspace serves any
+ * number of calls of any shapes whose moe_workspace_bytes(...) it covers,
+ * including calls replayed from a CUDA graph, as long as calls sharing a
+ * workspace are ordered on one stream.
  */
 #ifndef MOE_H_
 #define MOE_H_
@@ -85,6 +88,13 @@ typedef int32_t moe_status_t;
 #define MOE_ERR_CUDA (-4)
 #define MOE_ERR_TIMEOUT (-5)
 #define MOE_ERR_DEVICE_DATA (-6)
+
+/* Debug switches (moe_workspace_set_limits).  MOE_DEBUG_STARVE_FIRST_WAIT:
+ * the first warp of the row-block GEMV's gate/up kernel waits on a stage that
+ * no copy fills, so its bounded wait runs out and MOE_ERR_TIMEOUT is latched
+ * (the error path of a device-side wait, exercised without any fault); the
+ * call's output is then undefined.  For tests only. */
+#define MOE_DEBUG_STARVE_FIRST_WAIT 1u
 
 typedef struct moe_shape {
   int32_t T; /* tokens in the batch */
@@ -118,11 +128,17 @@ typedef struct moe_mxfp4_experts {
  * (the pages' quality mode, "ds4-ssd" README, "Experimental Pro Support":
  * --quality / --no-int8), with float32 accumulation.  On the CUDA-core path
  * for T <= 512 (the row-block GEMV, whose products run on f16 tensor-core
- * operands) the tokens enter as f16 (exact for 2^-17 <= |x| < 65520) and the
- * SwiGLU output h as the pair hi = f16(h), lo = f16(h - hi) (22 significant
- * bits); an |h| of 65520 or more latches MOE_ERR_DEVICE_DATA.  MXFP4: each
- * projection input row is quantised to MXFP4 in 32-element blocks first
- * (scale 2^(floor(log2 amax) - 2), round-to-nearest-even onto the E2M1 grid,
+ * operands) token row t enters as f16 values of x * 2^-s_t, its largest
+ * magnitude scaled into [1, 2) and 2^s_t applied to the sums: every bf16
+ * value within 2^-17 of its row's largest magnitude is exact, smaller ones
+ * carry an absolute error below 2^-25 of that magnitude.  The SwiGLU output h
+ * enters as the pair hi = f16(h 2^-e), lo = f16(h 2^-e - hi) with one power
+ * of two 2^e per 32 values (22 significant bits for every value within 2^-18
+ * of its block's largest magnitude, an absolute error below 2^-39 of it for
+ * the others).  A non-finite value in a token row makes that token's output
+ * non-finite.  MXFP4: each projection
+ * input row is quantised to MXFP4 in 32-element blocks first (scale
+ * 2^(floor(log2 amax) - 2), round-to-nearest-even onto the E2M1 grid,
  * saturating at +-6), as an accelerator path does. */
 #define MOE_ACT_EXACT 0
 #define MOE_ACT_MXFP4 1
@@ -135,6 +151,13 @@ MOE_API size_t moe_workspace_bytes(moe_shape_t shape, int32_t path, int32_t prec
 
 /* Zero a workspace before its first use (asynchronous memset on stream). */
 MOE_API moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Set, for later calls on ws (asynchronous, ordered on stream): the bound of
+ * every device-side wait in microseconds (0: the default of 2 s; a wait that
+ * runs out latches MOE_ERR_TIMEOUT and its kernel returns) and the debug
+ * switches (MOE_DEBUG_*, 0 for none). */
+MOE_API moe_status_t moe_workspace_set_limits(void* ws, uint32_t wait_us, uint32_t debug,
+                                              void* stream);
 
 /* Router, softmax, top-k and renormalisation.
  * logits[t,e] = sum_h x[t,h] W_r[e,h] + bias[e] in float32 (bias may be NULL);
@@ -197,8 +220,12 @@ MOE_API moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router,
  * the library until the process exits; a shape whose moe_workspace_bytes(...,
  * MOE_PATH_GEMV, ...) exceeds it returns MOE_ERR_WORKSPACE.  The first call on
  * a device looks up the array's device address (make it before any stream
- * capture).  Every call reuses the same array: calls that overlap on the GPU
- * race and must be ordered on one stream.  Inputs and outputs as for
+ * capture).  Every call reuses the same array, which keeps what the last call
+ * left there; each call clears the words it needs at zero itself.  Calls that
+ * overlap on the GPU race and must be ordered on one stream.  A device-side
+ * error (an expired wait, MOE_ERR_TIMEOUT) is latched in the array and stays
+ * there, for this and later calls on the device, until
+ * moe_get_error_static() reads it.  Inputs and outputs as for
  * moe_layer_forward; topk_idx_out / topk_w_out may be NULL. */
 MOE_API moe_status_t moe_layer_forward_static(const uint16_t* x, const float* w_router,
                                               const float* bias,
@@ -208,14 +235,22 @@ MOE_API moe_status_t moe_layer_forward_static(const uint16_t* x, const float* w_
                                               uint16_t* y, int32_t* topk_idx_out,
                                               float* topk_w_out, void* stream);
 
+/* moe_get_error() for moe_layer_forward_static on the current device:
+ * synchronise `stream`, return the first device-side error latched in the
+ * static scratch since the last read (MOE_OK if none) and clear it.  Allocates
+ * nothing. */
+MOE_API moe_status_t moe_get_error_static(void* stream);
+
 /* Quantise rows [rows, K] float32 to MXFP4 (codes [rows, K/2], scales
  * [rows, K/32]) with the MOE_ACT_MXFP4 rule above; K % 32 == 0. */
 MOE_API moe_status_t moe_act_quant_mxfp4(const float* in, int32_t rows, int32_t K,
                                  uint8_t* q_out, uint8_t* s_out, void* stream);
 
 /* Decode MXFP4 rows (codes [rows, K/2], scales [rows, K/32]) to float32
- * [rows, K] with the same in-register decode the FFN kernels use (E2M1 value
- * times 2^(scale-127); scale byte 255 gives NaN).  For tests and tools. */
+ * [rows, K] with the conversions the row-block GEMV uses (cvt e2m1x2 -> f16x2
+ * for the codes, cvt ue8m0x2 -> bf16x2 for the scales): E2M1 value times
+ * 2^(scale-127), scale byte 0 the subnormal 2^-127, byte 255 NaN.  For tests
+ * and tools. */
 MOE_API moe_status_t moe_decode_mxfp4(const uint8_t* q, const uint8_t* s, int32_t rows,
                               int32_t K, float* out, void* stream);
 

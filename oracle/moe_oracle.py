@@ -28,7 +28,7 @@ What the layer computes, and where the pages say so
 The pages print no formula for the router, softmax, top-k, SwiGLU or combine;
 the plainest reading is taken for each and written next to the function.
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings where the pages are silent (the CUDA library takes the same ones):
   R1 nibble order: byte b of a row holds element 2b in its low nibble and 2b+1
      in its high nibble; scale byte q covers elements 32q..32q+31 along the
      row's contiguous (input) dimension.

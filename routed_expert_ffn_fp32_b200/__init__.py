@@ -7,6 +7,6 @@ from . import moe  # noqa: F401
 from .moe import (  # noqa: F401
     EXPORTS, Experts, MoeError, load_library, make_workspace, moe_act_quant_mxfp4,
     moe_bucket, moe_combine, moe_decode_mxfp4, moe_expert_ffn_mxfp4, moe_get_error,
-    moe_layer_forward, moe_route_topk, moe_version, moe_workspace_bytes, moe_workspace_init,
-    shape_of,
+    moe_get_error_static, moe_layer_forward, moe_layer_forward_static, moe_route_topk,
+    moe_version, moe_workspace_bytes, moe_workspace_init, moe_workspace_set_limits, shape_of,
 )

@@ -144,6 +144,12 @@ moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
 }
 
+moe_status_t moe_workspace_set_limits(void* ws, uint32_t wait_us, uint32_t debug, void* stream) {
+  if (ws == nullptr || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_set_words(static_cast<uint32_t*>(ws) + 2, wait_us, debug,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_route_topk(const uint16_t* x, const float* w_router, const float* bias,
                             moe_shape_t shape, float* logits_out, int32_t* topk_idx,
                             float* topk_w, void* ws, size_t ws_bytes, void* stream) {
@@ -244,7 +250,11 @@ moe_status_t moe_expert_ffn_mxfp4(const moe_mxfp4_experts_t* experts,
   a.act_mxfp4 = precision == MOE_ACT_MXFP4;
   if (rp == MOE_PATH_GEMM) return cuda_status(launch_ffn_gemm(a, gemm_buffers(ws, L, shape.E), s));
   a.xh = at<uint16_t>(ws, L.xh);
-  e = launch_x_f16(x, shape.T, shape.H, a.act_mxfp4, at<uint16_t>(ws, L.xh), s);
+  a.xexp = at<uint8_t>(ws, L.xexp);
+  const bool lane = shape.T <= kLaneMaxT;
+  e = launch_x_f16(x, shape.T, shape.H, a.act_mxfp4, at<uint16_t>(ws, L.xh), at<uint8_t>(ws, L.xexp),
+                   lane ? at<uint32_t>(ws, L.lane_cnt) : nullptr,
+                   lane ? int(lane_cnt_words(shape, has_shared)) : 0, s);
   if (e != cudaSuccess) return cuda_status(e);
   return cuda_status(launch_gemv_path(a, ws, L, s));
 }
@@ -300,7 +310,12 @@ moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router, const f
   r.k = shape.k;
   if (rp == MOE_PATH_GEMV) {
     r.xh = at<uint16_t>(ws, L.xh);
+    r.xexp = at<uint8_t>(ws, L.xexp);
     r.act_mxfp4 = precision == MOE_ACT_MXFP4;
+    if (shape.T <= kLaneMaxT) {
+      r.cnt_clear = at<uint32_t>(ws, L.lane_cnt);
+      r.cnt_words = int(lane_cnt_words(shape, has_shared));
+    }
   }
   r.has_shared = has_shared;
   cudaError_t e;
@@ -310,7 +325,8 @@ moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router, const f
     e = launch_route_logits(r, false, s);
     if (e == cudaSuccess) e = launch_topk(r, s);
     if (e == cudaSuccess) e = launch_bucket(r, s);
-    if (e == cudaSuccess && r.xh != nullptr) e = launch_x_f16(x, shape.T, shape.H, r.act_mxfp4, r.xh, s);
+    if (e == cudaSuccess && r.xh != nullptr)
+      e = launch_x_f16(x, shape.T, shape.H, r.act_mxfp4, r.xh, r.xexp, r.cnt_clear, r.cnt_words, s);
   }
   if (e != cudaSuccess) return cuda_status(e);
 
@@ -333,6 +349,7 @@ moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router, const f
   a.has_shared = has_shared;
   a.act_mxfp4 = precision == MOE_ACT_MXFP4;
   a.xh = r.xh;
+  a.xexp = r.xexp;
   e = rp == MOE_PATH_GEMM ? launch_ffn_gemm(a, gemm_buffers(ws, L, shape.E), s)
                           : launch_gemv_path(a, ws, L, s);
   if (e == cudaSuccess)

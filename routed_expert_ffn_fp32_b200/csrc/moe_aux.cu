@@ -17,7 +17,8 @@ __global__ void __launch_bounds__(256) k_decode(const uint8_t* q, const uint8_t*
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= nblk) return;
   const uint4 c = *reinterpret_cast<const uint4*>(q + i * 16);
-  const float sc = e8m0_to_f32(s[i]);
+  // the scale through the same hardware ue8m0 conversion the row-block GEMV uses
+  const float sc = __uint_as_float(ue8m0x2_to_bf16x2(uint32_t(s[i])) << 16);
   const uint32_t w[4] = {c.x, c.y, c.z, c.w};
   float4* o = reinterpret_cast<float4*>(out + i * 32);
 #pragma unroll
@@ -67,7 +68,18 @@ __global__ void __launch_bounds__(256) k_act_quant(const float* in, long long nb
   s[i] = uint8_t(X + 127);
 }
 
+__global__ void k_set_words(uint32_t* words, uint32_t w0, uint32_t w1) {
+  pdl_wait();
+  pdl_trigger();
+  words[0] = w0;
+  words[1] = w1;
+}
+
 }  // namespace
+
+cudaError_t launch_set_words(uint32_t* words, uint32_t w0, uint32_t w1, cudaStream_t st) {
+  return launch_pdl(k_set_words, dim3(1), dim3(1), 0, st, words, w0, w1);
+}
 
 cudaError_t launch_decode(const uint8_t* q, const uint8_t* s, int rows, int K, float* out,
                           cudaStream_t st) {

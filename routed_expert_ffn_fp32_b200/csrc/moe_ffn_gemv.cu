@@ -212,9 +212,10 @@ constexpr int kGemvSmem = kWarps * kRingBytes + kPartBytes;
 template <int PHASE>
 struct PhaseCfg {
   static constexpr int NPROJ = PHASE == 0 ? 2 : 1;
-  // gate/up: token rows enter as f16 (exact for bf16 inputs); down: the
-  // float32 SwiGLU output enters as it is.
-  static constexpr int POL = PHASE == 0 ? kMixed : kF32x2;
+  // Both projections take their inputs as float32 (bf16 token rows and the
+  // float32 SwiGLU output are exact there, over the whole bf16 range), with
+  // the weights widened to float32 and packed float32 FMAs.
+  static constexpr int POL = kF32x2;
 };
 
 struct Worker {
@@ -368,8 +369,11 @@ __device__ void run_segment(const FfnArgs& a, const VExpert& ve, int r0, int r1,
   __syncwarp();
 }
 
+// Four CTAs per SM, or two where the float32 operand registers of BPL * RCMAX
+// blocks per lane would not fit the register budget of four.
 template <int PHASE, int BPL, int RCMAX>
-__global__ void __launch_bounds__(kThreads, 4) k_ffn_gemv(FfnArgs a, int KS, int fast_scales) {
+__global__ void __launch_bounds__(kThreads, BPL * RCMAX >= 4 ? 2 : 4)
+    k_ffn_gemv(FfnArgs a, int KS, int fast_scales) {
   extern __shared__ __align__(128) unsigned char smem[];
   pdl_wait();
   pdl_trigger();
@@ -493,22 +497,44 @@ __global__ void __launch_bounds__(256) k_combine(const float* partial, const flo
   *reinterpret_cast<uint2*>(y + size_t(t) * H + c) = out;
 }
 
-// bf16 token rows -> f16 (for callers that did not route through the router)
-__global__ void __launch_bounds__(256) k_x_f16(const uint16_t* x, int nblk, int act_mxfp4,
-                                               uint16_t* xh) {
+// bf16 token rows -> scaled f16 rows and their exponents (for calls that do
+// not route through the fused router): one warp per token row finds the
+// row's largest magnitude, then converts its 32-value blocks.  The grid also
+// zeroes the row-block GEMV's split-block counters.
+__global__ void __launch_bounds__(256) k_x_f16(const uint16_t* x, int T, int H, int act_mxfp4,
+                                               uint16_t* xh, uint8_t* xexp, uint32_t* cnt,
+                                               int cnt_words) {
   pdl_wait();
   pdl_trigger();
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nblk; i += gridDim.x * blockDim.x)
-    bf16_block_to_f16(x + size_t(i) * 32, xh + size_t(i) * 32, act_mxfp4 != 0);
+  const int lane = threadIdx.x & 31;
+  const int nthr = gridDim.x * blockDim.x;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < cnt_words; i += nthr) cnt[i] = 0u;
+  const int nwarps = nthr / 32;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) / 32; t < T; t += nwarps) {
+    const uint16_t* row = x + size_t(t) * H;
+    uint32_t m = 0;
+    for (int i = lane; i < H / 8; i += 32) m = bf16x8_absmax(__ldg(reinterpret_cast<const uint4*>(row) + i), m);
+    m = max(m & 0xffffu, m >> 16);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) m = max(m, __shfl_xor_sync(kFull, m, off));
+    const int sx = row_f16_exponent(m);
+    if (lane == 0) xexp[t] = uint8_t(sx + 127);
+    const float inv = exp2i(-sx);
+    for (int b = lane; b < H / 32; b += 32)
+      bf16_block_to_f16(row + size_t(b) * 32, xh + size_t(t) * H + size_t(b) * 32, act_mxfp4 != 0,
+                        inv);
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_x_f16(const uint16_t* x, int T, int H, int act_mxfp4, uint16_t* xh,
-                         cudaStream_t st) {
-  const int nblk = T * (H / 32);
-  const int grid = min(1024, (nblk + 255) / 256);
-  return launch_pdl(k_x_f16, dim3(grid), dim3(256), 0, st, x, nblk, act_mxfp4, xh);
+                         uint8_t* xexp, uint32_t* cnt_clear, int cnt_words, cudaStream_t st) {
+  const int by_rows = (T + 7) / 8;
+  const int by_cnt = (cnt_words + 255) / 256;
+  const int grid = max(1, min(1024, max(by_rows, by_cnt)));
+  return launch_pdl(k_x_f16, dim3(grid), dim3(256), 0, st, x, T, H, act_mxfp4, xh, xexp,
+                    cnt_clear, cnt_clear ? cnt_words : 0);
 }
 
 int gemv_grid() {

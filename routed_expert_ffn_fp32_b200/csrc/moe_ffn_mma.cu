@@ -24,19 +24,30 @@
 // a quad owns values 8c..8c+7, so the fragment's k order is a fixed
 // permutation of the block that B follows as well (one 16-byte load of a
 // token row per block and thread).  The two MMAs of a block start from zero
-// and the block's E8M0 scale (2^(s-127), per weight row) multiplies their sum
-// into the float32 accumulators: every product is exact (f16 x f16 fits a
-// float32) and the sums are float32, though the order of the additions inside
-// an MMA is the hardware's, not a scalar loop's.  Gate/up take the f16 token rows;
-// down takes h as a pair of f16 rows hi + lo (h to 22 significant bits), the
-// two columns of a token summed at the end.
+// and the block's E8M0 scale (decoded by the hardware ue8m0 conversion, so
+// byte 0 is 2^-127 and byte 255 NaN) multiplies their sum into the float32
+// accumulators: every product is exact (f16 x f16 fits a float32) and the sums
+// are float32, though the order of the additions inside an MMA is the
+// hardware's, not a scalar loop's.
+//
+// Operand range.  f16 holds magnitudes up to 65504, so the operands carry
+// powers of two: token row t enters as x * 2^-s_t (its largest magnitude in
+// [1, 2), s_t written with the f16 rows) and the gate/up sums are
+// multiplied by 2^s_t before the SwiGLU; the SwiGLU output h enters the down
+// projection as the pair hi = f16(h * 2^-e), lo = f16(h * 2^-e - hi) with one
+// exponent e per 32-value block of a row (its largest magnitude in
+// [2^14, 2^15)), applied to the block's MMA sums before the weight scale.
+// Every bf16 token value within 2^-17 of its row's largest magnitude is exact
+// and every h value within 2^-18 of its block's largest magnitude keeps 22
+// significant bits.
 //
 // Data movement.  Each warp keeps D slots of shared memory.  A slot holds the
 // 32 x 64-byte code box of an atom per projection, loaded by a TMA tile copy
 // (64-byte swizzle: the 4-byte fragment loads of the 32 lanes fall in distinct
 // banks), and the atom's 128 f16 values of each operand row (1-D bulk copies,
-// one per row).  Scale bytes come in TMA boxes of 32 rows x 16 bytes (four
-// atoms) where a row's scale bytes are a multiple of 16, else one 4-byte
+// one per row; the down projection adds the 16 bytes of block exponents of
+// four atoms per token).  Scale bytes come in TMA boxes of 32 rows x 16 bytes
+// (four atoms) where a row's scale bytes are a multiple of 16, else one 4-byte
 // cp.async per row and atom.  All complete on the slot's mbarrier; the copy
 // for stage j + D is issued as soon as stage j has been consumed.  Weight
 // loads carry an L2 evict-first policy (read once per call).
@@ -50,8 +61,9 @@
 // expert output row).  A row block split between warps is finished
 // deterministically by the warp that holds its first atom (see run_pass).
 //
-// Every wait is bounded (globaltimer); on expiry the kernel latches
-// MOE_ERR_TIMEOUT, lets its in-flight copies land and returns.
+// Every wait is bounded (globaltimer; the limit is a workspace word); on
+// expiry the kernel latches MOE_ERR_TIMEOUT, lets its in-flight copies land
+// and returns.
 #include <cuda.h>
 
 #include "moe_internal.cuh"
@@ -72,24 +84,22 @@ constexpr int kAtomCode = kAtomVals / 2; // code bytes of a row per atom
 constexpr int kBlk = kAtomVals / 32;     // scale blocks per atom
 constexpr int kBox = 32 * kAtomCode;     // one projection's 32-row code box
 constexpr int kXRow = kAtomVals * 2;     // one f16 operand row of an atom
-constexpr unsigned long long kLWaitNs = 2000000000ull;
+constexpr int kXExp = 16;                // block exponents of one h row, four atoms
 constexpr int kPfxMax = kLanePfxMax;     // per-expert table entries (virtual experts + 1)
 constexpr int kEntMax = 512;             // bucket entries staged in shared memory
-constexpr int kOwnMax = 32;              // contributors listed per owned split block
-// f16 range: larger magnitudes round to infinity
-constexpr float kF16Limit = 65520.f;
+constexpr int kOwnMax = 32;              // contributors listed per split block
+constexpr int kSlotF = kRMax * 2 * 32;   // floats of one split-block slot
 
 // Shared memory: [barriers][pass prefix][cost prefix][tokens][plan][offsets]
-// [scan scratch][entries], then from the next 1024-byte boundary per warp
-// its D stage slots (code boxes, operand rows) and its NSCE scale entries.
+// [scan scratch][entries][contributor lists][token exponents], then from the
+// next 1024-byte boundary per warp its D stage slots (code boxes, operand
+// rows), its NSCE scale entries and (down) its D block-exponent chunks.
 // A scale entry holds [NPROJ][32 rows][16 bytes]: the scale bytes of four
 // atoms of each row (one TMA box per projection), or of one atom (cp.async)
 // when a row's scale bytes are not a multiple of 16.
-// Gate/up runs 10 warps (its scale entries are twice the size), down 11;
-// two to six slots per warp and 8 to 11 warps measured the same.
 template <int NPROJ>
 struct LaneCfg {
-  static constexpr int NW = NPROJ == 2 ? 10 : 11;  // warps per CTA
+  static constexpr int NW = kLaneWarps;            // warps per CTA
   static constexpr int THREADS = 32 * NW;
   static constexpr int D = 3;                      // slots per warp
   static constexpr int CODE = NPROJ * kBox;                     // code bytes per slot
@@ -97,21 +107,23 @@ struct LaneCfg {
   static constexpr int SLOT = CODE + XROWS * kXRow;
   static constexpr int SCE = NPROJ * 32 * 16;                   // one scale entry
   static constexpr int NSCE = 3;                                // scale entries per warp
-  static constexpr int WARP_BYTES = D * SLOT + NSCE * SCE;
+  static constexpr int EXPB = NPROJ == 1 ? D * kRMax * kXExp : 0;
+  static constexpr int WARP_BYTES = (D * SLOT + NSCE * SCE + EXPB + 511) / 512 * 512;
   static constexpr int SLOTS = NW * D;
-  static constexpr int HEAD =
-      SLOTS * 8 + 5 * kPfxMax * 4 + 2 * NW * 4 + kEntMax * 4 + NW * kOwnMax * 4;
+  static constexpr int HEAD = SLOTS * 8 + 5 * kPfxMax * 4 + 2 * NW * 4 + kEntMax * 4 +
+                              NW * kOwnMax * 4 + kLaneMaxT;
   static constexpr int SMEM = 1024 + HEAD + NW * WARP_BYTES;
   static_assert(SLOT % 512 == 0 && SCE % 512 == 0, "64-byte swizzle boxes start on 512 bytes");
-  static_assert(NW <= kLaneWarps, "split-block slots are sized for kLaneWarps warps");
   static_assert(D <= NSCE, "a scale entry outlives the stages in flight");
+  static_assert(2 * kRMax <= 16, "operand-row copies use lanes below 16");
 };
 static_assert(LaneCfg<2>::SMEM + 1024 <= 227 * 1024, "shared memory per block");
 static_assert(LaneCfg<1>::SMEM + 1024 <= 227 * 1024, "shared memory per block");
 
 struct LaneArgs {
-  float* part;    // split-block partial sums, one slot per warp: [warp][kRMax][NPROJ][32]
-  uint32_t* cnt;  // split-block atom counts of the contributors, one per row block
+  float* part;    // split-block partial sums, one slot per warp: [grid warp][kSlotF]
+  uint32_t* cnt;  // split-block atom counts of the contributors, one per row block, zero at the
+                  // call's start
   int NA;         // atoms per row: K / 128
   int RB;         // row blocks per projection: ROWS / 32
   int sbox;       // scale bytes by TMA boxes of 4 atoms (K / 32 a multiple of 16)
@@ -137,13 +149,14 @@ __device__ __forceinline__ bool lane_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Lane 0 waits for the phase (bounded); the outcome is warp-uniform.
-__device__ __forceinline__ bool lane_wait(uint32_t bar, uint32_t parity, int* err, int where) {
+// Lane 0 waits for the phase (bounded by limit_ns); the outcome is warp-uniform.
+__device__ __forceinline__ bool lane_wait(uint32_t bar, uint32_t parity, int* err, int where,
+                                          unsigned long long limit_ns) {
   int ok = 1;
   if ((threadIdx.x & 31) == 0 && !lane_try(bar, parity)) {
     const unsigned long long t0 = lane_now();
     while (!lane_try(bar, parity)) {
-      if (lane_now() - t0 > kLWaitNs) {
+      if (lane_now() - t0 > limit_ns) {
         latch_error(err, MOE_ERR_TIMEOUT, where);
         ok = 0;
         break;
@@ -152,16 +165,8 @@ __device__ __forceinline__ bool lane_wait(uint32_t bar, uint32_t parity, int* er
   }
   return __shfl_sync(kFull, ok, 0) != 0;
 }
-__device__ __forceinline__ void lane_tma(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                         uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-// The same with an L2 cache policy (weights: read once, evict first, so the
-// stream does not push out the instructions and the small hot data).
+// TMA tile copy with an L2 cache policy (weights: read once, evict first, so
+// the stream does not push out the instructions and the small hot data).
 __device__ __forceinline__ void lane_tma_hint(uint32_t dst, const CUtensorMap* map, int x, int y,
                                               uint32_t bar, uint64_t policy) {
   asm volatile(
@@ -186,7 +191,6 @@ __device__ __forceinline__ void lane_bulk(uint32_t dst, const void* src, uint32_
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
-
 // d += A B for one m16n8k16 tile, f16 inputs, f32 accumulators.
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -196,14 +200,18 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// E8M0 byte J of a word of four scale bytes as the float 2^(s-127).  Byte 0
-// reads as 0 (its products lie below float32's normal range; they are lost in
-// any nonzero float32 sum) and byte 255 as infinity (the block's products are
-// then not finite, like the NaN the format assigns it).
+// Four E8M0 bytes (the blocks of one atom of one row, or four biased block
+// exponents) as bf16 powers of two: bytes 0, 1 in lo, bytes 2, 3 in hi.
+struct Pow4 {
+  uint32_t lo, hi;
+};
+__device__ __forceinline__ Pow4 pow4_of(uint32_t w) {
+  return {ue8m0x2_to_bf16x2(w), ue8m0x2_to_bf16x2(w >> 16)};
+}
 template <int J>
-__device__ __forceinline__ float scale_f32(uint32_t w) {
-  const uint32_t bits = (J < 3 ? (w << (23 - 8 * J)) : (w >> 1)) & 0x7f800000u;
-  return __uint_as_float(bits);
+__device__ __forceinline__ float pow_at(const Pow4& p) {
+  const uint32_t v = J < 2 ? p.lo : p.hi;
+  return __uint_as_float((J & 1) ? (v & 0xffff0000u) : (v << 16));
 }
 
 // MXFP4 round trip of v with the block scale exponent X (OCP MX v1.0: RNE
@@ -213,6 +221,17 @@ __device__ __forceinline__ float mx_round(float v, int X) {
   uint32_t h2[4];
   e2m1x8_to_f16x2(byte, h2);
   return f16x2_to_f32x2(h2[0]).x * exp2i(X);
+}
+
+// Exponent e of the power of two that brings a 32-value block of h with
+// largest magnitude amax into [2^14, 2^15) for its f16 pair: clamped to
+// [-126, 113]; 0 for a zero or non-finite block.
+__device__ __forceinline__ int h_block_exponent(float amax) {
+  const uint32_t bits = __float_as_uint(amax);
+  if (bits == 0u || bits >= 0x7f800000u) return 0;
+  const int field = int(bits >> 23);
+  const int e = field == 0 ? -126 : field - 127 - 14;
+  return e < -126 ? -126 : e;
 }
 
 // ------------------------------------------------------ fragment mapping ---
@@ -227,13 +246,15 @@ __device__ __forceinline__ int frag_row(int g, int mt, int i) { return mt * 16 +
 // ------------------------------------------------------- routing metadata ---
 // The routing arrays every lookup of the kernel needs, preloaded into shared
 // memory in one round of independent loads: plan (active experts), offsets
-// (bucket starts) and, for batches of at most kEntMax pairs, the bucket
-// entries themselves (larger batches read them from global memory).
+// (bucket starts), the token rows' scale exponents and, for batches of at
+// most kEntMax pairs, the bucket entries themselves (larger batches read them
+// from global memory).
 struct Meta {
-  const int* plan;  // [0] active experts nA, [1 + v] expert id of virtual expert v
-  const int* off;   // bucket offsets [E + 1]
-  const int* ent;   // bucket entries (pair indices), shared or global memory
-  const int* rv;    // tokens of virtual expert v
+  const int* plan;     // [0] active experts nA, [1 + v] expert id of virtual expert v
+  const int* off;      // bucket offsets [E + 1]
+  const int* ent;      // bucket entries (pair indices), shared or global memory
+  const int* rv;       // tokens of virtual expert v
+  const uint8_t* xe;   // s_t + 127 of token t
   int nA, nV, T, k;
   __device__ __forceinline__ int expert(int v) const { return v < nA ? plan[1 + v] : -1; }
   // output row (pair index, or T*k + r for the shared expert) of bucket row r
@@ -301,6 +322,16 @@ struct LanePart {
   const int* rv;    // tokens of v, [nV]
   int nV, RBNA, B, total;
 
+  __device__ __forceinline__ void init(const int* p, const int* c, const int* r, int n, int rbna,
+                                       int nwarps) {
+    pfx = p;
+    cpfx = c;
+    rv = r;
+    nV = n;
+    RBNA = rbna;
+    total = c[n] * rbna;
+    B = (total + nwarps - 1) / nwarps;
+  }
   __device__ __forceinline__ int atom_at(int g) const {
     const int c = min(total, g * B);
     if (c >= total) return pfx[nV] * RBNA;
@@ -334,29 +365,33 @@ struct LaneWarp {
   const CUtensorMap* smaps; // scale maps, same order (TMA scale boxes)
   unsigned char* codes;     // this warp's D code slots
   unsigned char* scales;    // this warp's NSCE scale entries
+  unsigned char* exps;      // (down) this warp's D block-exponent chunks [D][kRMax][16]
   int ri;                   // scale entry of the last TMA scale load
   uint32_t sring;           // scale entry of the stage in slot d: bits 2d, 2d + 1
   uint64_t* full;           // this warp's D barriers
   const int* pfx;           // pass prefix of the virtual experts
   LanePart part;
   int nV, K, ROWS, nb, lane;
-  int gw, A0, A1;           // this warp's index in the grid and atom range
+  int gw;                   // this warp's index in the grid
+  unsigned long long wait_ns;
+  bool starve;              // debug: stage 0 gets no copies (its wait runs out)
   LaneIt nxt;               // next stage to load
   int jc, ji;               // stages consumed / issued (ji counts empty tail slots)
-  int jv;                   // stages issued with a copy in flight
+  uint32_t pend, ppar;      // slots with copies in flight, and their phase parities
   int iv, ipass;            // (virtual expert, pass) of the cached operand rows below
   int irows;                // f16 operand rows of that pass (tokens, or tokens x 2)
   const unsigned char* ixsrc;  // lane < irows: the start of its operand row
+  const unsigned char* iesrc;  // (down) lane 16 + t < 16 + tokens: token t's block exponents
   // per segment being loaded: first atom, TMA row, maps, this lane's scale rows
   int iseg, iy;
   const CUtensorMap* imap;
   const CUtensorMap* ismap;
   const uint8_t* isrc[NPROJ];
   int islot;                // ji % D
-  // prologue of the down projection: operand-row copies deferred until the
+  // prologue of the down projection: operand copies deferred until the
   // SwiGLU rows of the previous kernel are complete
   const void* dsrc[C::D];
-  uint32_t ddst[C::D], dfb[C::D];
+  uint32_t ddst[C::D], dfb[C::D], dsz[C::D];
   int cslot;                // jc % D
   uint32_t cpar;            // (jc / D) & 1
   // the other contributors of the split row block this warp owns at the end
@@ -379,17 +414,21 @@ struct LaneWarp {
       const int t0 = ipass * kRMax;
       const int R = min(kRMax, m->rv[iv] - t0);
       ixsrc = nullptr;
+      iesrc = nullptr;
       if constexpr (PHASE == 0) {
         irows = R;
         if (lane < R)
           ixsrc = reinterpret_cast<const unsigned char*>(a->xh + size_t(m->token(iv, t0 + lane)) * a->H);
       } else {
-        // h row of a pair: I f16 values hi, then I f16 values lo
+        // h row of a pair: I f16 values hi, I f16 values lo, block exponents
         irows = 2 * R;
+        const size_t pitch = h_pitch(size_t(a->I));
+        const unsigned char* hb = reinterpret_cast<const unsigned char*>(a->h);
         if (lane < 2 * R)
-          ixsrc = reinterpret_cast<const unsigned char*>(a->h) +
-                  size_t(m->out_row(iv, t0 + (lane >> 1))) * (size_t(a->I) * 4) +
+          ixsrc = hb + size_t(m->out_row(iv, t0 + (lane >> 1))) * pitch +
                   size_t(lane & 1) * (size_t(a->I) * 2);
+        if (lane >= 16 && lane < 16 + R)
+          iesrc = hb + size_t(m->out_row(iv, t0 + lane - 16)) * pitch + size_t(a->I) * 4;
       }
     }
     const size_t row = size_t(nxt.rb * 32 + lane);
@@ -406,9 +445,9 @@ struct LaneWarp {
   }
 
   // Load stage ji (if any) into slot ji % D: the code boxes, the atom's values
-  // of the pass's operand rows, and the rows' scale bytes.  DJ >= 0: a
-  // prologue stage (ji == DJ) whose operand-row copy is kept for
-  // flush_deferred().
+  // of the pass's operand rows (down: and their block exponents), and the
+  // rows' scale bytes.  DJ >= 0: a prologue stage (ji == DJ) whose operand
+  // copies are kept for flush_deferred().
   template <int DJ = -1>
   __device__ __forceinline__ void issue() {
     if (nxt.valid) {
@@ -429,63 +468,83 @@ struct LaneWarp {
         ent = ri;
       }
       sring = (sring & ~(3u << (2 * islot))) | (uint32_t(ent) << (2 * islot));
-      const uint32_t sdst = lsm(scales + size_t(ent) * C::SCE);
-      // this slot's previous contents were read through the generic proxy
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      if (lane == 0) {
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(fb),
-                     "r"(uint32_t(NPROJ * kBox) + uint32_t(irows) * kXRow +
-                         (sload ? uint32_t(C::SCE) : 0u))
-                     : "memory");
-        const uint64_t pol = evict_first_policy();
-#pragma unroll
-        for (int pj = 0; pj < NPROJ; ++pj)
-          lane_tma_hint(dst + pj * kBox, imap + pj, atom * kAtomCode, iy, fb, pol);
-        if (sload)
+      const bool skip = starve && ji == 0;
+      if (!skip) {
+        const uint32_t sdst = lsm(scales + size_t(ent) * C::SCE);
+        // this slot's previous contents were read through the generic proxy
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (lane == 0) {
+          const uint32_t ebytes = PHASE == 1 ? uint32_t(irows / 2) * kXExp : 0u;
+          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(fb),
+                       "r"(uint32_t(NPROJ * kBox) + uint32_t(irows) * kXRow + ebytes +
+                           (sload ? uint32_t(C::SCE) : 0u))
+                       : "memory");
+          const uint64_t pol = evict_first_policy();
 #pragma unroll
           for (int pj = 0; pj < NPROJ; ++pj)
-            lane_tma_hint(sdst + pj * (C::SCE / NPROJ), ismap + pj, 16 * (atom >> 2), iy, fb, pol);
-      }
-      __syncwarp();
-      const void* xsrc = lane < irows ? ixsrc + size_t(kbase) * 2 : nullptr;
-      if constexpr (DJ >= 0) {
-        dsrc[DJ] = xsrc;
-        ddst[DJ] = dst + C::CODE + lane * kXRow;
-        dfb[DJ] = fb;
-      } else if (xsrc != nullptr) {
-        lane_bulk(dst + C::CODE + lane * kXRow, xsrc, kXRow, fb);
-      }
-      if (!l->sbox) {
+            lane_tma_hint(dst + pj * kBox, imap + pj, atom * kAtomCode, iy, fb, pol);
+          if (sload)
 #pragma unroll
-        for (int pj = 0; pj < NPROJ; ++pj)
-          lane_cp4(sdst + pj * (C::SCE / NPROJ) + lane * 16, isrc[pj] + atom * kBlk);
-        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(fb) : "memory");
+            for (int pj = 0; pj < NPROJ; ++pj)
+              lane_tma_hint(sdst + pj * (C::SCE / NPROJ), ismap + pj, 16 * (atom >> 2), iy, fb,
+                            pol);
+        }
+        __syncwarp();
+        // operand copy of this lane: an operand row, or (down) a token's
+        // block exponents of this group of four atoms
+        const void* xsrc = nullptr;
+        uint32_t xdst = 0, xsz = 0;
+        if (ixsrc != nullptr) {
+          xsrc = ixsrc + size_t(kbase) * 2;
+          xdst = dst + C::CODE + lane * kXRow;
+          xsz = kXRow;
+        } else if (PHASE == 1 && iesrc != nullptr) {
+          xsrc = iesrc + size_t(atom >> 2) * kXExp;
+          xdst = lsm(exps + size_t(islot) * (kRMax * kXExp) + (lane - 16) * kXExp);
+          xsz = kXExp;
+        }
+        if constexpr (DJ >= 0) {
+          dsrc[DJ] = xsrc;
+          ddst[DJ] = xdst;
+          dsz[DJ] = xsz;
+          dfb[DJ] = fb;
+        } else if (xsrc != nullptr) {
+          lane_bulk(xdst, xsrc, xsz, fb);
+        }
+        if (!l->sbox) {
+#pragma unroll
+          for (int pj = 0; pj < NPROJ; ++pj)
+            lane_cp4(sdst + pj * (C::SCE / NPROJ) + lane * 16, isrc[pj] + atom * kBlk);
+          asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(fb) : "memory");
+        }
+        pend |= 1u << islot;
+        ppar = (ppar & ~(1u << islot)) | (((uint32_t(ji) / C::D) & 1u) << islot);
+      } else if constexpr (DJ >= 0) {
+        dsrc[DJ] = nullptr;
       }
       it_next(nxt, *l, pfx, nV);
-      ++jv;
-    }
-    else if constexpr (DJ >= 0) {
+    } else if constexpr (DJ >= 0) {
       dsrc[DJ] = nullptr;
     }
     if (++islot == C::D) islot = 0;
     ++ji;
   }
 
-  // The deferred operand-row copies of the prologue stages.
+  // The deferred operand copies of the prologue stages.
   __device__ __forceinline__ void flush_deferred() {
 #pragma unroll
     for (int j = 0; j < C::D; ++j)
-      if (dsrc[j] != nullptr) lane_bulk(ddst[j], dsrc[j], kXRow, dfb[j]);
+      if (dsrc[j] != nullptr) lane_bulk(ddst[j], dsrc[j], dsz[j], dfb[j]);
   }
 
   // After a timeout: let the copies already issued land (bounded) so the
   // block's shared memory outlives them.
   __device__ void drain() {
     if (lane == 0) {
-      for (int j = jc; j < jv; ++j) {
+      for (int d = 0; d < C::D; ++d) {
+        if (!((pend >> d) & 1u)) continue;
         const unsigned long long t0 = lane_now();
-        while (!lane_try(lsm(&full[j % C::D]), uint32_t(j / C::D) & 1u) &&
-               lane_now() - t0 < 100000000ull) {
+        while (!lane_try(lsm(&full[d]), (ppar >> d) & 1u) && lane_now() - t0 < 100000000ull) {
         }
       }
     }
@@ -528,11 +587,9 @@ __device__ __forceinline__ void tile_block(const unsigned char* box, int wofs, c
   mma16816(d, h0[2], h1[2], h0[3], h1[3], b.z, b.w);
 }
 
-// acc (rows g, g + 8 of a tile) += d * the rows' scales of block J.
-template <int J>
-__device__ __forceinline__ void scale_acc(float (&acc)[4], const float (&d)[4], uint32_t s0,
-                                          uint32_t s1) {
-  const float f0 = scale_f32<J>(s0), f1 = scale_f32<J>(s1);
+// acc (rows g, g + 8 of a tile) += d * (f0, f1).
+__device__ __forceinline__ void scale_acc(float (&acc)[4], const float (&d)[4], float f0,
+                                          float f1) {
   acc[0] = fmaf(d[0], f0, acc[0]);
   acc[1] = fmaf(d[1], f0, acc[1]);
   acc[2] = fmaf(d[2], f1, acc[2]);
@@ -543,8 +600,7 @@ __device__ __forceinline__ void scale_acc(float (&acc)[4], const float (&d)[4], 
 // tokens (the slot's f16 token rows).
 template <int J>
 __device__ __forceinline__ void gateup_block(const unsigned char* slot, const FragOfs& f,
-                                             const uint32_t (&sw)[2][2][2],
-                                             float (&acc)[2][2][4]) {
+                                             const Pow4 (&sw)[2][2][2], float (&acc)[2][2][4]) {
   using C = LaneCfg<2>;
   const uint4 b = *reinterpret_cast<const uint4*>(slot + C::CODE + f.x + 64 * J);
 #pragma unroll
@@ -553,13 +609,13 @@ __device__ __forceinline__ void gateup_block(const unsigned char* slot, const Fr
     for (int mt = 0; mt < 2; ++mt) {
       float d[4];
       tile_block(slot + p * kBox + mt * 16 * kAtomCode, f.w[J], b, d);
-      scale_acc<J>(acc[p][mt], d, sw[p][mt][0], sw[p][mt][1]);
+      scale_acc(acc[p][mt], d, pow_at<J>(sw[p][mt][0]), pow_at<J>(sw[p][mt][1]));
     }
 }
 // sc: the stage's scale words in its scale entry ([projection][32 rows][16 B]).
 __device__ __forceinline__ void stage_gateup(const unsigned char* slot, const unsigned char* sc,
                                              const FragOfs& f, float (&acc)[2][2][4]) {
-  uint32_t sw[2][2][2];  // scale words: [projection][tile][row g / g + 8]
+  Pow4 sw[2][2][2];  // scales: [projection][tile][row g / g + 8]
 #pragma unroll
   for (int p = 0; p < 2; ++p)
 #pragma unroll
@@ -567,17 +623,19 @@ __device__ __forceinline__ void stage_gateup(const unsigned char* slot, const un
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh)
         sw[p][mt][hh] =
-            *reinterpret_cast<const uint32_t*>(sc + p * 512 + f.s + (mt * 16 + hh * 8) * 16);
+            pow4_of(*reinterpret_cast<const uint32_t*>(sc + p * 512 + f.s + (mt * 16 + hh * 8) * 16));
   gateup_block<0>(slot, f, sw, acc);
   gateup_block<1>(slot, f, sw, acc);
   gateup_block<2>(slot, f, sw, acc);
   gateup_block<3>(slot, f, sw, acc);
 }
 
-// Phase 1: down rows for NT column tiles of (token, hi/lo) operand rows.
+// Phase 1: down rows for NT column tiles of (token, hi/lo) operand rows; the
+// weight scale of a block times the token's block exponent of h.
 template <int J, int NT>
 __device__ __forceinline__ void down_block(const unsigned char* slot, const FragOfs& f,
-                                           const uint32_t (&sw)[2][2], float (&acc)[NT][2][4]) {
+                                           const Pow4 (&sw)[2][2], const Pow4 (&ew)[NT],
+                                           float (&acc)[NT][2][4]) {
   using C = LaneCfg<1>;
   uint4 b[NT];
 #pragma unroll
@@ -591,28 +649,41 @@ __device__ __forceinline__ void down_block(const unsigned char* slot, const Frag
     uint32_t h0[4], h1[4];
     e2m1x8_to_f16x2(w0, h0);
     e2m1x8_to_f16x2(w1, h1);
+    const float f0 = pow_at<J>(sw[mt][0]), f1 = pow_at<J>(sw[mt][1]);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       float d[4] = {0.f, 0.f, 0.f, 0.f};
       mma16816(d, h0[0], h1[0], h0[1], h1[1], b[nt].x, b[nt].y);
       mma16816(d, h0[2], h1[2], h0[3], h1[3], b[nt].z, b[nt].w);
-      scale_acc<J>(acc[nt][mt], d, sw[mt][0], sw[mt][1]);
+      // the block exponent of h first, then the weight scale: each product
+      // overflows only where the unscaled term would
+      const float fe = pow_at<J>(ew[nt]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d[i] *= fe;
+      scale_acc(acc[nt][mt], d, f0, f1);
     }
   }
 }
+// ex: the stage's block-exponent chunks [kRMax tokens][16 bytes]; atom & 3
+// selects the atom's four bytes.
 template <int NT>
 __device__ __forceinline__ void stage_down(const unsigned char* slot, const unsigned char* sc,
-                                           const FragOfs& f, float (&acc)[NT][2][4]) {
-  uint32_t sw[2][2];
+                                           const unsigned char* ex, int atom, const FragOfs& f,
+                                           int c, float (&acc)[NT][2][4]) {
+  Pow4 sw[2][2];
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh)
-      sw[mt][hh] = *reinterpret_cast<const uint32_t*>(sc + f.s + (mt * 16 + hh * 8) * 16);
-  down_block<0, NT>(slot, f, sw, acc);
-  down_block<1, NT>(slot, f, sw, acc);
-  down_block<2, NT>(slot, f, sw, acc);
-  down_block<3, NT>(slot, f, sw, acc);
+      sw[mt][hh] = pow4_of(*reinterpret_cast<const uint32_t*>(sc + f.s + (mt * 16 + hh * 8) * 16));
+  Pow4 ew[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+    ew[nt] = pow4_of(*reinterpret_cast<const uint32_t*>(ex + (nt * 4 + c) * kXExp + 4 * (atom & 3)));
+  down_block<0, NT>(slot, f, sw, ew, acc);
+  down_block<1, NT>(slot, f, sw, ew, acc);
+  down_block<2, NT>(slot, f, sw, ew, acc);
+  down_block<3, NT>(slot, f, sw, ew, acc);
 }
 
 // ---------------------------------------------------------------- results ---
@@ -662,46 +733,58 @@ __device__ __forceinline__ void collect(const float (&acc)[PHASE == 0 ? 2 : NT][
 }
 
 // Epilogue of a finished row block of virtual expert v, pass tokens t0 ..
-// t0 + R - 1 (all lanes call: the MXFP4 rounding of h reduces over the
+// t0 + R - 1 (all lanes call: the block exponent of h reduces over the
 // block's 32 rows with shuffles).
 template <int PHASE, int NT>
 __device__ __forceinline__ void block_store(const FfnArgs& a, const Meta& m, int v, int t0, int R,
-                                            int row0, int lane, const BlockVals<PHASE, NT>& o) {
+                                            int rb, int lane, const BlockVals<PHASE, NT>& o) {
   const int g = lane >> 2, c = lane & 3;
+  const int row0 = rb * 32;
   if constexpr (PHASE == 0) {
-    // h for tokens 2c and 2c + 1: [tile][element]
+    // the gate/up sums of tokens 2c and 2c + 1 back to the token rows' scale,
+    // then h: [tile][element]
+    float sx[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int t = 2 * c + q;
+      sx[q] = t < R ? __uint_as_float(uint32_t(m.xe[m.token(v, t0 + t)]) << 23) : 1.f;
+    }
     float hv[8];
 #pragma unroll
     for (int n = 0; n < 8; ++n) {
-      const float gt = o.v[n], up = o.v[8 + n];
+      const float gt = o.v[n] * sx[n & 1], up = o.v[8 + n] * sx[n & 1];
       hv[n] = gt / (1.f + expf(-gt)) * up;
     }
-    if (a.act_mxfp4) {
-      // one MXFP4 block along I per token: the 32 rows of this block, held by
-      // the eight threads of quad column c
+    const size_t pitch = h_pitch(size_t(a.I));
+    unsigned char* hbase = reinterpret_cast<unsigned char*>(a.h);
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        float amax = fmaxf(fmaxf(fabsf(hv[q]), fabsf(hv[2 + q])), fmaxf(fabsf(hv[4 + q]), fabsf(hv[6 + q])));
+    for (int q = 0; q < 2; ++q) {
+      // one 32-value block along I per token: the 32 rows of this block,
+      // held by the eight threads of quad column c
+      float amax = fmaxf(fmaxf(fabsf(hv[q]), fabsf(hv[2 + q])), fmaxf(fabsf(hv[4 + q]), fabsf(hv[6 + q])));
 #pragma unroll
-        for (int off = 4; off <= 16; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
+      for (int off = 4; off <= 16; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
+      if (a.act_mxfp4) {
         const int X = mx_scale_exponent(amax);
 #pragma unroll
         for (int n = q; n < 8; n += 2) hv[n] = mx_round(hv[n], X);
       }
-    }
-    uint16_t* hbase = reinterpret_cast<uint16_t*>(a.h);
-#pragma unroll
-    for (int n = 0; n < 8; ++n) {
-      const int t = 2 * c + (n & 1);
+      const int eb = h_block_exponent(amax);
+      const float inv = exp2i(-eb);
+      const int t = 2 * c + q;
       if (t < R) {
-        const float h = hv[n];
-        if (fabsf(h) >= kF16Limit && fabsf(h) <= 3.4028235e38f) latch_error(a.err, MOE_ERR_DEVICE_DATA, 431);
-        const __half hi = __float2half_rn(h);
-        const __half lo = __float2half_rn(h - __half2float(hi));
-        uint16_t* hr = hbase + size_t(m.out_row(v, t0 + t)) * (size_t(a.I) * 2);
-        const int row = row0 + frag_row(g, n >> 2, n & 3);
-        hr[row] = __half_as_ushort(hi);
-        hr[a.I + row] = __half_as_ushort(lo);
+        unsigned char* hr = hbase + size_t(m.out_row(v, t0 + t)) * pitch;
+        uint16_t* hi16 = reinterpret_cast<uint16_t*>(hr);
+#pragma unroll
+        for (int n = q; n < 8; n += 2) {
+          const float hs = hv[n] * inv;
+          const __half hi = __float2half_rn(hs);
+          const __half lo = __float2half_rn(hs - __half2float(hi));
+          const int row = row0 + frag_row(g, n >> 2, n & 3);
+          hi16[row] = __half_as_ushort(hi);
+          hi16[a.I + row] = __half_as_ushort(lo);
+        }
+        if (g == 0) hr[size_t(a.I) * 4 + rb] = uint8_t(eb + 127);
       }
     }
   } else {
@@ -724,7 +807,7 @@ __device__ __forceinline__ void block_store(const FfnArgs& a, const Meta& m, int
 // without waiting.  The owner, at the end of its range, waits (bounded) until
 // the count is complete, adds the contributors' slots after its own sums in
 // atom order (the same order whichever warps share the block) and applies the
-// epilogue; it then clears the counter for the next call.
+// epilogue; it then clears the counter.
 template <int PHASE, int NT>
 __device__ bool run_pass(LaneWarp<PHASE>& W, LaneIt& cur, const FragOfs& f) {
   constexpr int NPROJ = LaneWarp<PHASE>::NPROJ;
@@ -738,7 +821,6 @@ __device__ bool run_pass(LaneWarp<PHASE>& W, LaneIt& cur, const FragOfs& f) {
   const int R = min(kRMax, m.rv[v] - t0);
   const int seg0 = cur.seg0, nst = cur.seg1 - cur.seg0;
   const int blk = cur.blk;
-  const int row0 = rb * 32;
   float acc[PHASE == 0 ? 2 : NT][2][4];
 #pragma unroll
   for (int p = 0; p < (PHASE == 0 ? 2 : NT); ++p)
@@ -749,14 +831,15 @@ __device__ bool run_pass(LaneWarp<PHASE>& W, LaneIt& cur, const FragOfs& f) {
 
   for (int s = 0; s < nst; ++s) {
     const int d = W.cslot;
-    if (!lane_wait(lsm(&W.full[d]), W.cpar, a.err, 410)) return false;
+    if (!lane_wait(lsm(&W.full[d]), W.cpar, a.err, 410, W.wait_ns)) return false;
     const unsigned char* slot = W.codes + size_t(d) * C::SLOT;
     const int atom = cur.a - blk * l.NA;
     const unsigned char* sc = W.scales + size_t((W.sring >> (2 * d)) & 3u) * C::SCE +
                               (l.sbox ? 4 * (atom & 3) : 0);
     if constexpr (PHASE == 0) stage_gateup(slot, sc, f, acc);
-    else stage_down<NT>(slot, sc, f, acc);
+    else stage_down<NT>(slot, sc, W.exps + size_t(d) * (kRMax * kXExp), atom, f, c, acc);
     __syncwarp();
+    W.pend &= ~(1u << d);
     ++W.jc;
     if (++W.cslot == C::D) {
       W.cslot = 0;
@@ -769,15 +852,14 @@ __device__ bool run_pass(LaneWarp<PHASE>& W, LaneIt& cur, const FragOfs& f) {
   BlockVals<PHASE, NT> o;
   collect<PHASE, NT>(acc, o);
   constexpr int NV = BlockVals<PHASE, NT>::N;
-  constexpr int SLOTF = kRMax * NPROJ * 32;  // floats per contributor slot
   const int B0 = blk * l.NA;
   if (seg0 == B0 && nst == l.NA) {  // whole row block: final values
-    block_store<PHASE, NT>(a, m, v, t0, R, row0, lane, o);
+    block_store<PHASE, NT>(a, m, v, t0, R, rb, lane, o);
     return true;
   }
   if (seg0 != B0) {
     // contributor: partial sums into this warp's slot, then count them in
-    float* slotp = l.part + size_t(W.gw) * SLOTF;
+    float* slotp = l.part + size_t(W.gw) * kSlotF;
 #pragma unroll
     for (int n = 0; n < NV; ++n) {
       int t, row, p;
@@ -785,10 +867,10 @@ __device__ bool run_pass(LaneWarp<PHASE>& W, LaneIt& cur, const FragOfs& f) {
       if (t < R) slotp[(t * NPROJ + p) * 32 + row] = o.v[n];
     }
     // Count in with a release-ordered add from lane 31: it issues no copies
-    // (the operand rows take at most 16 lanes, the tensor copies lane 0), so
-    // its release waits only for the slot stores, which __syncwarp orders
-    // before it, and not for this warp's stage loads in flight (a full
-    // sequentially consistent fence would).
+    // (the operand rows and block exponents take lanes below 24, the tensor
+    // copies lane 0), so its release waits only for the slot stores, which
+    // __syncwarp orders before it, and not for this warp's stage loads in
+    // flight (a full sequentially consistent fence would).
     __syncwarp();
     if (lane == 31)
       asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(l.cnt + blk), "r"(uint32_t(nst))
@@ -805,7 +887,7 @@ __device__ bool run_pass(LaneWarp<PHASE>& W, LaneIt& cur, const FragOfs& f) {
       const unsigned long long t_0 = lane_now();
       do {
         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(got) : "l"(l.cnt + blk) : "memory");
-        if (got != want && lane_now() - t_0 > kLWaitNs) {
+        if (got != want && lane_now() - t_0 > W.wait_ns) {
           latch_error(a.err, MOE_ERR_TIMEOUT, 420);
           ok = 0;
           break;
@@ -821,7 +903,7 @@ __device__ bool run_pass(LaneWarp<PHASE>& W, LaneIt& cur, const FragOfs& f) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const bool use = q0 + q < W.on;
-        const float* sp = l.part + size_t(use ? W.osid[q0 + q] : 0) * SLOTF;
+        const float* sp = l.part + size_t(use ? W.osid[q0 + q] : 0) * kSlotF;
 #pragma unroll
         for (int n = 0; n < NV; ++n) {
           int t, row, p;
@@ -862,7 +944,7 @@ __device__ bool run_pass(LaneWarp<PHASE>& W, LaneIt& cur, const FragOfs& f) {
       float val[4][NV];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float* sp = l.part + size_t(sid[q] < 0 ? 0 : sid[q]) * SLOTF;
+        const float* sp = l.part + size_t(sid[q] < 0 ? 0 : sid[q]) * kSlotF;
 #pragma unroll
         for (int n = 0; n < NV; ++n) {
           int t, row, p;
@@ -877,7 +959,7 @@ __device__ bool run_pass(LaneWarp<PHASE>& W, LaneIt& cur, const FragOfs& f) {
           for (int n = 0; n < NV; ++n) o.v[n] += val[q][n];
     }
   }
-  block_store<PHASE, NT>(a, m, v, t0, R, row0, lane, o);
+  block_store<PHASE, NT>(a, m, v, t0, R, rb, lane, o);
   __syncwarp();
   if (lane == 0) *reinterpret_cast<volatile uint32_t*>(l.cnt + blk) = 0u;
   return true;
@@ -911,6 +993,7 @@ __global__ void __launch_bounds__(LaneCfg<PHASE == 0 ? 2 : 1>::THREADS, 1)
   int* s_wsum = s_off + kPfxMax;                                  // [kLW][2]
   int* s_ent = s_wsum + 2 * kLW;                                  // [kEntMax]
   int* s_own = s_ent + kEntMax;                                   // [kLW][kOwnMax]
+  uint8_t* s_xe = reinterpret_cast<uint8_t*>(s_own + kLW * kOwnMax);  // [kLaneMaxT]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
 
@@ -921,6 +1004,7 @@ __global__ void __launch_bounds__(LaneCfg<PHASE == 0 ? 2 : 1>::THREADS, 1)
   W.smaps = maps.s;
   W.codes = codes + size_t(warp) * C::WARP_BYTES;
   W.scales = W.codes + C::D * C::SLOT;
+  W.exps = W.scales + C::NSCE * C::SCE;
   W.ri = C::NSCE - 1;
   W.sring = 0;
   W.full = bars + warp * C::D;
@@ -937,19 +1021,25 @@ __global__ void __launch_bounds__(LaneCfg<PHASE == 0 ? 2 : 1>::THREADS, 1)
   if constexpr (PHASE == 0) pdl_wait();
   pdl_trigger();
 
-  // Routing metadata: one round of independent loads into shared memory.
+  // Routing metadata and the workspace's wait limit and debug switches: one
+  // round of independent loads into shared memory / registers.
   const int npairs = a.T * a.k;
   const bool ent_smem = npairs <= kEntMax;
+  const unsigned wait_us = __ldg(reinterpret_cast<const unsigned*>(a.err) + 2);
+  const unsigned debug = __ldg(reinterpret_cast<const unsigned*>(a.err) + 3);
   for (int i = tid; i < a.E + 2; i += kLThreads) s_plan[i] = __ldg(a.plan + i);
   for (int i = tid; i <= a.E; i += kLThreads) s_off[i] = __ldg(a.offsets + i);
   if (ent_smem)
     for (int i = tid; i < npairs; i += kLThreads) s_ent[i] = __ldg(a.entries + i);
+  if constexpr (PHASE == 0)
+    for (int i = tid; i < a.T; i += kLThreads) s_xe[i] = __ldg(a.xexp + i);
   __syncthreads();
   Meta meta;
   meta.plan = s_plan;
   meta.off = s_off;
   meta.ent = ent_smem ? s_ent : a.entries;
   meta.rv = s_rv;
+  meta.xe = s_xe;
   meta.nA = s_plan[0];
   meta.nV = meta.nA + (a.has_shared ? 1 : 0);
   meta.T = a.T;
@@ -961,14 +1051,17 @@ __global__ void __launch_bounds__(LaneCfg<PHASE == 0 ? 2 : 1>::THREADS, 1)
   W.nb = W.K / 32;
   W.nV = meta.nV;
   W.lane = lane;
-  W.jc = W.ji = W.jv = 0;
+  W.jc = W.ji = 0;
+  W.pend = W.ppar = 0;
   W.iv = -1;
   W.ipass = -1;
   W.irows = 0;
   W.ixsrc = nullptr;
+  W.iesrc = nullptr;
   W.iseg = -1;
   W.islot = W.cslot = 0;
   W.cpar = 0;
+  W.wait_ns = (wait_us ? wait_us : kDefaultWaitUs) * 1000ull;
 
   // Per virtual expert: tokens, passes and cost; prefix sums over the
   // experts (two entries per thread).
@@ -1021,28 +1114,20 @@ __global__ void __launch_bounds__(LaneCfg<PHASE == 0 ? 2 : 1>::THREADS, 1)
     __syncthreads();
   }
   W.pfx = s_pfx;
-  W.part.pfx = s_pfx;
-  W.part.cpfx = s_cpfx;
-  W.part.rv = s_rv;
-  W.part.nV = W.nV;
-  W.part.RBNA = l.RB * l.NA;
-  W.part.total = s_cpfx[W.nV] * W.part.RBNA;
-  {
-    const int NW = gridDim.x * kLW;
-    W.part.B = (W.part.total + NW - 1) / NW;
-  }
+  const int NWtot = gridDim.x * kLW;
+  W.part.init(s_pfx, s_cpfx, s_rv, W.nV, l.RB * l.NA, NWtot);
 
   W.gw = blockIdx.x * kLW + warp;
-  W.A0 = W.part.atom_at(W.gw);
-  W.A1 = W.part.atom_at(W.gw + 1);
-  if (W.A0 >= W.A1) {
+  const int A0 = W.part.atom_at(W.gw), A1 = W.part.atom_at(W.gw + 1);
+  W.starve = (debug & MOE_DEBUG_STARVE_FIRST_WAIT) != 0 && PHASE == 0 && W.gw == 0;
+  if (A0 >= A1) {
     if constexpr (PHASE == 1) pdl_wait();
     return;
   }
 
   LaneIt cur;
-  it_begin(cur, W.A0, W.A1, l, W.pfx, W.nV);
-  it_begin(W.nxt, W.A0, W.A1, l, W.pfx, W.nV);
+  it_begin(cur, A0, A1, l, W.pfx, W.nV);
+  it_begin(W.nxt, A0, A1, l, W.pfx, W.nV);
   if constexpr (PHASE == 1) {
     static_assert(C::D <= 4, "prologue");
     W.template issue<0>();
@@ -1060,13 +1145,14 @@ __global__ void __launch_bounds__(LaneCfg<PHASE == 0 ? 2 : 1>::THREADS, 1)
   W.on = -1;
   W.osid = s_own + warp * kOwnMax;
   {
-    const int lb0 = (W.A1 - 1) / l.NA * l.NA;  // first atom of the last row block
-    if (lb0 >= W.A0 && W.A1 - lb0 < l.NA) {
+    const int NA = l.NA;
+    const int lb0 = (A1 - 1) / NA * NA;  // first atom of the last row block
+    if (lb0 >= A0 && A1 - lb0 < NA) {
       // lanes look up the next warps' first atoms in parallel; the
       // contributors are the non-empty ones among them, in order
-      const int B1 = lb0 + l.NA;
+      const int B1 = lb0 + NA;
       int n = 0, w = W.gw + 1;
-      int at = W.A1;  // first atom of warp w
+      int at = A1;  // first atom of warp w
       bool done = false;
       while (!done && n < kOwnMax) {
         const int nx = W.part.atom_at(w + 1 + lane);  // first atom of warp w + 1 + lane
@@ -1126,7 +1212,7 @@ bool lane_supported(const moe_shape_t& s) {
 cudaError_t launch_ffn_lane(const FfnArgs& a, float* lane_part, uint32_t* lane_cnt,
                             cudaStream_t st) {
   moe_shape_t s{a.T, a.H, a.I, a.E, a.k};
-  if (!lane_supported(s) || a.xh == nullptr) return cudaErrorNotSupported;
+  if (!lane_supported(s) || a.xh == nullptr || a.xexp == nullptr) return cudaErrorNotSupported;
   LaneMaps g{}, d{};
   const uint64_t HB = uint64_t(a.H) / 2, IB = uint64_t(a.I) / 2;
   bool ok = make_tma_map_u8_box(&g.m[0], a.ex.gq, HB, uint64_t(a.E) * a.I, kAtomCode, 32) &&

@@ -20,14 +20,8 @@ constexpr unsigned kFull = 0xffffffffu;
 // GEMV), CTAs (one per SM, at most), warps per CTA, tokens per pass.
 constexpr int kLaneMaxT = 512;
 constexpr int kLaneMaxCtas = 160;
-#ifndef MOE_LANE_WARPS
-#define MOE_LANE_WARPS 11
-#endif
-#ifndef MOE_LANE_RMAX
-#define MOE_LANE_RMAX 8
-#endif
-constexpr int kLaneWarps = MOE_LANE_WARPS;
-constexpr int kLaneRMax = MOE_LANE_RMAX;
+constexpr int kLaneWarps = 10;
+constexpr int kLaneRMax = 8;
 // Per-virtual-expert tables of the row-block GEMV's work split (tokens, passes
 // before v, cost units before v, plan, offsets): virtual experts + 1 entries.
 constexpr int kLanePfxMax = 258;
@@ -35,8 +29,12 @@ constexpr int kLanePfxMax = 258;
 // ---------------------------------------------------------------------------
 // Workspace layout.  Every region starts on a 256-byte boundary.
 // ---------------------------------------------------------------------------
+// Words of the error region: [0] status, [1] detail, [2] wait limit in
+// microseconds (0: kDefaultWaitUs), [3] debug switches (MOE_DEBUG_*).
+constexpr unsigned kDefaultWaitUs = 2000000u;
+
 struct WsLayout {
-  size_t err;       // int32[16]: [0] status, [1] detail
+  size_t err;       // int32[16]: status, detail, wait limit, debug switches
   size_t counters;  // uint32[16]: arrival counters, zero between calls
   size_t logits;    // f32 [T, E]
   size_t idx;       // i32 [T, k]
@@ -45,13 +43,16 @@ struct WsLayout {
   size_t offsets;   // i32 [E + 1]
   size_t entries;   // i32 [T * k]
   size_t plan;      // i32 [E + 2]: [0] active experts, [1..] their ids (ascending)
-  size_t xh;        // f16 [T, H]  token rows as f16 (MXFP4-rounded in that mode)
-  size_t h;         // [T*k + S*T] rows of 4I bytes: SwiGLU output by pair index (f32, or f16 hi then f16 lo in the row-block GEMV)
+  size_t xh;        // f16 [T, H]  token rows as f16, row t scaled by 2^-s_t (MXFP4-rounded first in that mode)
+  size_t xexp;      // u8 [T]      s_t + 127
+  size_t h;         // [T*k + S*T] rows of h_pitch(I) bytes: SwiGLU output by pair index (f32 [I] on
+                    //             the K-split GEMV; f16 hi [I], f16 lo [I], block exponents on the
+                    //             row-block GEMV)
   size_t partial;   // f32 [T*k + S*T, H]   expert output rows (by pair index)
   // row-block GEMV (T <= kLaneMaxT)
   size_t lane_part;  // f32 [warps][kLaneRMax][2][32]  split row-block partial sums
-  size_t lane_cnt;   // u32 [row blocks]  split row-block atom counts: zero between calls,
-                     //     every call leaves them zero
+  size_t lane_cnt;   // u32 [row blocks]  split row-block atom counts, cleared by the kernel that
+                     //     writes the f16 token rows, before every call's GEMV
   // tensor-core path only
   size_t xq, xs;    // u8 [rows, H/2], [rows, H/32]  MXFP4 token rows, bucket order
   size_t hq, hs;    // u8 [rows, I/2], [rows, I/32]  MXFP4 SwiGLU rows, bucket order
@@ -61,6 +62,21 @@ struct WsLayout {
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 __host__ __device__ inline size_t align_up16(size_t v) { return (v + 15) & ~size_t(15); }
+
+// Bytes of one h row: f16 hi [I], f16 lo [I], then one exponent byte per
+// 32-value block, padded to 16 bytes (at least the I float32 values of the
+// K-split GEMV).
+__host__ __device__ inline size_t h_pitch(size_t I) { return 4 * I + align_up16(I / 32); }
+
+// Split-block counters of the row-block GEMV: one per row block of the larger
+// phase and per pass (at most one pass per virtual expert plus one per
+// kLaneRMax rows).
+inline size_t lane_cnt_words(const moe_shape_t& s, int has_shared) {
+  const size_t rows = size_t(s.T) * s.k + (has_shared ? s.T : 0);
+  const size_t passes = size_t(s.E) + 1 + (rows + kLaneRMax - 1) / kLaneRMax;
+  const size_t rb0 = size_t(s.I) / 32, rb1 = size_t(s.H) / 32;
+  return passes * (rb0 > rb1 ? rb0 : rb1);
+}
 
 inline WsLayout ws_layout(const moe_shape_t& s, int has_shared, int gemm) {
   WsLayout L{};
@@ -78,14 +94,12 @@ inline WsLayout ws_layout(const moe_shape_t& s, int has_shared, int gemm) {
   L.entries = take(T * k * 4);
   L.plan = take((E + 2) * 4);
   L.xh = take(T * H * 2);
-  L.h = take(rows * I * 4);
+  L.xexp = take(T);
+  L.h = take(rows * h_pitch(I));
   L.partial = take(rows * H * 4);
   const bool lane = T <= size_t(kLaneMaxT);
   L.lane_part = take(lane ? size_t(kLaneMaxCtas) * kLaneWarps * kLaneRMax * 2 * 32 * 4 : 0);
-  // passes: at most one per virtual expert plus one per kLaneRMax rows
-  const size_t passes = E + 1 + (rows + kLaneRMax - 1) / kLaneRMax;
-  const size_t rb0 = I / 32, rb1 = H / 32;  // row blocks of the two phases
-  L.lane_cnt = take(lane ? passes * (rb0 > rb1 ? rb0 : rb1) * 4 : 0);
+  L.lane_cnt = take(lane ? lane_cnt_words(s, has_shared) * 4 : 0);
   if (gemm) {
     L.xq = take(rows * H / 2);
     L.xs = take(rows * H / 32);
@@ -204,9 +218,47 @@ __device__ __forceinline__ float exp2i(int e) {
   return e >= -126 ? __uint_as_float(uint32_t(e + 127) << 23) : __uint_as_float(0x00400000u);
 }
 
-// 32 bf16 values -> 32 f16 values (exact for |v| >= 2^-17 and |v| <= 65504);
-// with mx the block is first rounded through MXFP4 (OCP scale, RNE, saturate).
-__device__ __forceinline__ void bf16_block_to_f16(const uint16_t* src, uint16_t* dst, bool mx) {
+// Exponent s of the power-of-two scale of a token row's f16 copy, from the
+// row's largest bf16 magnitude (bits with the sign cleared): the row is stored
+// as x * 2^-s with its largest magnitude in [1, 2).  Every element down to
+// 2^-17 of that magnitude keeps its 8 significant bits (f16 subnormals start
+// at 2^-24), and no product of a weight with a scaled value exceeds twice the
+// weight, so the scaled sums overflow float32 only where sums of the weights'
+// magnitudes would.  s lies in [-126, 127]; a row of zeros, or one holding an
+// infinity or NaN, gets s = 0.
+__device__ __forceinline__ int row_f16_exponent(uint32_t amax_bf16_bits) {
+  if (amax_bf16_bits == 0u || amax_bf16_bits >= 0x7f80u) return 0;
+  const int field = int(amax_bf16_bits >> 7);  // bf16 exponent field; 0 for subnormals
+  return field == 0 ? -126 : field - 127;
+}
+
+// Largest magnitude of 8 bf16 values (16 bytes), as bf16 bits with the sign
+// cleared, folded into m (per-halfword unsigned max).
+__device__ __forceinline__ uint32_t bf16x8_absmax(const uint4& v, uint32_t m) {
+  m = __vmaxu2(m, v.x & 0x7fff7fffu);
+  m = __vmaxu2(m, v.y & 0x7fff7fffu);
+  m = __vmaxu2(m, v.z & 0x7fff7fffu);
+  m = __vmaxu2(m, v.w & 0x7fff7fffu);
+  return m;
+}
+
+// Two E8M0 scale bytes (low 16 bits of w) -> two bf16 powers of two
+// 2^(s-127) (low byte -> low half).  The conversion keeps the format's special
+// values: byte 0 is the subnormal 2^-127, byte 255 is NaN.
+__device__ __forceinline__ uint32_t ue8m0x2_to_bf16x2(uint32_t w) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo;\n\tmov.b32 {lo, _}, %1;\n\tcvt.rn.bf16x2.ue8m0x2 %0, lo;\n\t}"
+      : "=r"(r)
+      : "r"(w));
+  return r;
+}
+
+// 32 bf16 values -> 32 f16 values of v * inv, inv = 2^-s from
+// row_f16_exponent (exact for every element within 2^-17 of the row's largest
+// magnitude); with mx the block is first rounded through MXFP4 (OCP scale,
+// RNE, saturate) in float32.
+__device__ __forceinline__ void bf16_block_to_f16(const uint16_t* src, uint16_t* dst, bool mx,
+                                                  float inv) {
   float f[32];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -223,13 +275,13 @@ __device__ __forceinline__ void bf16_block_to_f16(const uint16_t* src, uint16_t*
 #pragma unroll
     for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(f[j]));
     const int X = mx_scale_exponent(amax);
-    const float inv = exp2i(-X), sc = exp2i(X);
+    const float qinv = exp2i(-X > 127 ? 127 : -X), sc = exp2i(X);
 #pragma unroll
     for (int j = 0; j < 32; j += 8) {
       uint32_t byte4 = 0;
 #pragma unroll
       for (int b = 0; b < 4; ++b)
-        byte4 |= f32x2_to_e2m1x2(f[j + 2 * b] * inv, f[j + 2 * b + 1] * inv) << (8 * b);
+        byte4 |= f32x2_to_e2m1x2(f[j + 2 * b] * qinv, f[j + 2 * b + 1] * qinv) << (8 * b);
       uint32_t h2[4];
       e2m1x8_to_f16x2(byte4, h2);
 #pragma unroll
@@ -243,10 +295,10 @@ __device__ __forceinline__ void bf16_block_to_f16(const uint16_t* src, uint16_t*
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     uint4 o;
-    o.x = f32x2_to_f16x2(f[8 * q + 0], f[8 * q + 1]);
-    o.y = f32x2_to_f16x2(f[8 * q + 2], f[8 * q + 3]);
-    o.z = f32x2_to_f16x2(f[8 * q + 4], f[8 * q + 5]);
-    o.w = f32x2_to_f16x2(f[8 * q + 6], f[8 * q + 7]);
+    o.x = f32x2_to_f16x2(f[8 * q + 0] * inv, f[8 * q + 1] * inv);
+    o.y = f32x2_to_f16x2(f[8 * q + 2] * inv, f[8 * q + 3] * inv);
+    o.z = f32x2_to_f16x2(f[8 * q + 4] * inv, f[8 * q + 5] * inv);
+    o.w = f32x2_to_f16x2(f[8 * q + 6] * inv, f[8 * q + 7] * inv);
     *reinterpret_cast<uint4*>(dst + 8 * q) = o;
   }
 }
@@ -265,8 +317,11 @@ struct ExpertPtrs {
 
 struct RouteArgs {
   const uint16_t* x;
-  uint16_t* xh;       // optional: f16 copy of x written by the router (decode path)
+  uint16_t* xh;       // optional: scaled f16 copy of x written by the router (decode path)
+  uint8_t* xexp;      // with xh: per-row scale exponents s_t + 127
   int act_mxfp4;      // round xh through MXFP4 first
+  uint32_t* cnt_clear;  // with xh: the row-block GEMV's split-block counters, zeroed here
+  int cnt_words;
   const float* w_router;
   const float* bias;
   float* logits;
@@ -286,7 +341,8 @@ struct FfnArgs {
   ExpertPtrs ex;
   ExpertPtrs sh;  // shared expert (n = 1) when has_shared
   const uint16_t* x;
-  const uint16_t* xh;   // f16 token rows [T, H] (decode path)
+  const uint16_t* xh;   // scaled f16 token rows [T, H] (decode path)
+  const uint8_t* xexp;  // their scale exponents s_t + 127 [T]
   const int32_t* offsets;
   const int32_t* entries;
   const int32_t* plan;
@@ -371,8 +427,10 @@ cudaError_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t st);
 cudaError_t launch_ffn_lane(const FfnArgs& a, float* lane_part, uint32_t* lane_cnt,
                             cudaStream_t st);
 bool lane_supported(const moe_shape_t& s);
+// Scaled f16 token rows and their exponents for the row-block GEMV; also zeroes
+// cnt_words split-block counters at cnt_clear (may be 0 / nullptr).
 cudaError_t launch_x_f16(const uint16_t* x, int T, int H, int act_mxfp4, uint16_t* xh,
-                         cudaStream_t st);
+                         uint8_t* xexp, uint32_t* cnt_clear, int cnt_words, cudaStream_t st);
 
 struct GemmBuffers {
   uint8_t* xq;
@@ -388,6 +446,8 @@ cudaError_t launch_combine(const float* partial, const float* w, int T, int H, i
                            int has_shared, uint16_t* y, cudaStream_t st);
 cudaError_t launch_act_quant(const float* in, int rows, int K, uint8_t* q, uint8_t* s,
                              cudaStream_t st);
+// words[0] = w0, words[1] = w1 (one thread; ordered on the stream).
+cudaError_t launch_set_words(uint32_t* words, uint32_t w0, uint32_t w1, cudaStream_t st);
 cudaError_t launch_decode(const uint8_t* q, const uint8_t* s, int rows, int K, float* out,
                           cudaStream_t st);
 

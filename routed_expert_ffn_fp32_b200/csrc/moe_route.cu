@@ -319,6 +319,7 @@ __device__ int bucket_warp(const int32_t* idx, int npairs, int E, int32_t* count
 template <int TT>
 __global__ void __launch_bounds__(kRouteThreads) k_route_logits(RouteArgs a, int fuse_tail) {
   extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ int s_exp[TT];
   pdl_wait();
   pdl_trigger();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -327,6 +328,19 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_logits(RouteArgs a, int
   const int nt = min(TT, a.T - t0);
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);                  // [TT][H] bf16
   float* red = reinterpret_cast<float*>(smem + size_t(TT) * H * 2);  // [8][TT]
+  const int e = blockIdx.x * 2 + (warp >> 2);
+  const int quarter = warp & 3;
+  const int qlen = H / 4;  // multiple of 8
+  const float* wrow = a.w_router + size_t(e < a.E ? e : 0) * H + quarter * qlen;
+  // the first eight float4 of this lane's router row go out before the token
+  // rows are staged, so the two loads overlap
+  float4 wv[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int c = lane * 4 + 128 * j;
+    wv[j] = (e < a.E && c < qlen) ? __ldg(reinterpret_cast<const float4*>(wrow + c))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   // stage the token rows (16-byte vectors; H % 32 == 0)
   {
     const int vec_per_row = H / 8;
@@ -334,34 +348,53 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_logits(RouteArgs a, int
     uint4* dst = reinterpret_cast<uint4*>(xs);
     for (int i = tid; i < nt * vec_per_row; i += kRouteThreads) dst[i] = __ldg(src + i);
   }
+  if (a.cnt_clear != nullptr) {
+    const int nthr = gridDim.x * gridDim.y * kRouteThreads;
+    for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * kRouteThreads + tid; i < a.cnt_words;
+         i += nthr)
+      a.cnt_clear[i] = 0u;
+  }
   __syncthreads();
   if (a.xh != nullptr) {
-    // f16 copy of the token rows for the expert GEMV: this token tile's
-    // 32-value blocks spread over the CTAs of the tile row, one per thread
+    // scale exponent of each token row of the tile (one warp per token)
+    if (warp < nt) {
+      uint32_t m = 0;
+      const uint4* row = reinterpret_cast<const uint4*>(xs + size_t(warp) * H);
+      for (int i = lane; i < H / 8; i += 32) m = bf16x8_absmax(row[i], m);
+      m = max(m & 0xffffu, m >> 16);
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) m = max(m, __shfl_xor_sync(kFull, m, off));
+      if (lane == 0) {
+        const int sx = row_f16_exponent(m);
+        s_exp[warp] = sx;
+        if (blockIdx.x == 0) a.xexp[t0 + warp] = uint8_t(sx + 127);
+      }
+    }
+    __syncthreads();
+    // scaled f16 copy of the token rows for the expert GEMV: this token
+    // tile's 32-value blocks spread over the CTAs of the tile row, one per
+    // thread
     const int nblk = nt * (H / 32);
     for (int i = blockIdx.x * kRouteThreads + tid; i < nblk; i += gridDim.x * kRouteThreads) {
       const int t = i / (H / 32), b = i % (H / 32);
       bf16_block_to_f16(xs + size_t(t) * H + 32 * b, a.xh + size_t(t0 + t) * H + 32 * b,
-                        a.act_mxfp4 != 0);
+                        a.act_mxfp4 != 0, exp2i(-s_exp[t]));
     }
   }
-  const int e = blockIdx.x * 2 + (warp >> 2);
-  const int quarter = warp & 3;
-  const int qlen = H / 4;  // multiple of 8
   float acc[TT];
 #pragma unroll
   for (int t = 0; t < TT; ++t) acc[t] = 0.f;
   if (e < a.E) {
-    const float* wrow = a.w_router + size_t(e) * H + quarter * qlen;
     const uint16_t* xq = xs + quarter * qlen;
     // eight float4 loads in flight per lane before the arithmetic on them
     for (int base = lane * 4; base < qlen; base += 128 * 8) {
-      float4 wv[8];
+      if (base != lane * 4) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int c = base + 128 * j;
-        wv[j] = c < qlen ? __ldg(reinterpret_cast<const float4*>(wrow + c))
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < 8; ++j) {
+          const int c = base + 128 * j;
+          wv[j] = c < qlen ? __ldg(reinterpret_cast<const float4*>(wrow + c))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
 #pragma unroll
       for (int j = 0; j < 8; ++j) {

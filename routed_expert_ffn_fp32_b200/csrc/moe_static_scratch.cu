@@ -18,12 +18,14 @@
 // allocating routine.
 //
 // All calls share the one array and it keeps whatever the previous call left
-// there; each call clears the words that must start at zero (the arrival
-// counter and the error word) with an asynchronous memset on its stream.  Two
-// calls whose work overlaps on the GPU (different streams, no ordering between
-// them) race on the array and corrupt each other's results.  The router makes
-// every expert index itself, so no device-side data error can arise; there is
-// no error word for the caller to read.
+// there.  Each call zeroes the arrival counter of the router with an
+// asynchronous memset on its stream; the kernels clear the rest of the scratch
+// they rely on (the row-block GEMV's split-block counters) at the start of
+// every call, so calls of different shapes may follow one another.  Two calls
+// whose work overlaps on the GPU (different streams, no ordering between
+// them) race on the array and corrupt each other's results.  A device-side
+// wait that runs out latches MOE_ERR_TIMEOUT in the array's error word, which
+// no call clears: moe_get_error_static() reads and clears it.
 #include <mutex>
 
 #include "moe_internal.cuh"
@@ -73,12 +75,19 @@ extern "C" moe_status_t moe_layer_forward_static(const uint16_t* x, const float*
   void* scratch = static_scratch_address();
   if (scratch == nullptr) return MOE_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the error word and the arrival counter sit in front of the logits region
-  const size_t zero_bytes = ws_layout(shape, shared != nullptr, 0).logits;
-  if (cudaMemsetAsync(scratch, 0, zero_bytes, s) != cudaSuccess) {
+  // the router's arrival counter (the error word in front of it stays latched
+  // until moe_get_error_static reads it)
+  const WsLayout L = ws_layout(shape, shared != nullptr, 0);
+  if (cudaMemsetAsync(static_cast<unsigned char*>(scratch) + L.counters, 0, 64, s) != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
   return moe_layer_forward(x, w_router, bias, experts, shared, shape, MOE_PATH_GEMV, precision, y,
                            topk_idx_out, topk_w_out, scratch, kStaticScratchBytes, stream);
+}
+
+extern "C" moe_status_t moe_get_error_static(void* stream) {
+  void* scratch = static_scratch_address();
+  if (scratch == nullptr) return MOE_ERR_CUDA;
+  return moe_get_error(scratch, stream);
 }

@@ -32,12 +32,14 @@ MOE_PATH_GEMM = 2
 MOE_ACT_EXACT = 0
 MOE_ACT_MXFP4 = 1
 
+MOE_DEBUG_STARVE_FIRST_WAIT = 1
+
 #: every symbol include/moe.h declares
 EXPORTS = (
     "moe_workspace_bytes", "moe_workspace_init", "moe_route_topk", "moe_bucket",
     "moe_expert_ffn_mxfp4", "moe_combine", "moe_layer_forward", "moe_act_quant_mxfp4",
     "moe_decode_mxfp4", "moe_get_error", "moe_status_string", "moe_version",
-    "moe_layer_forward_static",
+    "moe_layer_forward_static", "moe_get_error_static", "moe_workspace_set_limits",
 )
 
 
@@ -88,6 +90,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "moe_act_quant_mxfp4": (i32, [vp, i32, i32, vp, vp, vp]),
         "moe_decode_mxfp4": (i32, [vp, vp, i32, i32, vp, vp]),
         "moe_get_error": (i32, [vp, vp]),
+        "moe_get_error_static": (i32, [vp]),
+        "moe_workspace_set_limits": (i32, [vp, ctypes.c_uint32, ctypes.c_uint32, vp]),
         "moe_status_string": (ctypes.c_char_p, [i32]),
         "moe_version": (ctypes.c_char_p, []),
     }
@@ -243,6 +247,15 @@ def moe_decode_mxfp4(q, s, K, out, stream=None):
 
 def moe_get_error(ws, stream=None) -> int:
     return int(load_library().moe_get_error(_p(ws), _s(stream)))
+
+
+def moe_get_error_static(stream=None) -> int:
+    return int(load_library().moe_get_error_static(_s(stream)))
+
+
+def moe_workspace_set_limits(ws, wait_us: int = 0, debug: int = 0, stream=None):
+    _check(load_library().moe_workspace_set_limits(_p(ws), wait_us, debug, _s(stream)),
+           "moe_workspace_set_limits")
 
 
 def moe_version() -> str:

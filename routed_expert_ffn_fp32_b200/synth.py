@@ -11,7 +11,11 @@ encoded blocks, each block of the output picked uniformly from the pool: every
 block has the distribution of an encoded N(0, std) block while generation
 stays a few seconds per GB.
 
-Workloads (sizes as on the pages' DeepSeek-V4-Flash layers):
+Workloads (the decode64 shape is the 64-expert, top-2 model of the ainews.cool
+"antirez ds4 DeepSeek Metal inference" page; the fine-grained shape stands for
+the 284B DeepSeek-V4-Flash layer of the pawin.top ds4 guide and the ds4-ssd
+README, with its shared expert; the pages print no per-layer dimensions, so
+H, I and E are readings):
   tiny          H 256,  I 128,  E 8,   k 2, T 4,   router N(0,.05), no bias
   decode64      H 4096, I 1408, E 64,  k 2, T 1|5, router N(0,.02), no bias
   finegrained   H 4096, I 2048, E 256, k 8, T 1|5, shared expert, Zipf s=1.0 bias

@@ -13,8 +13,8 @@ import torch
 import oracle as O
 from routed_expert_ffn_fp32_b200 import build, moe, synth
 
-from helpers import (TOL_W, TOL_Y, bits_np, check_routing, dev_layer, gpu_layer, rel_l2,
-                     route_depth, to_dev_bits)
+from helpers import (TOL_W, TOL_Y, bits_np, check_routing, check_y, dev_layer, gpu_layer,
+                     rel_l2, route_depth, to_dev_bits)
 
 pytestmark = pytest.mark.gpu
 
@@ -92,10 +92,20 @@ def test_route_topk(name, T):
     bound = d * u / (1 - d * u) * (np.abs(xf) @ np.abs(W_r.astype(np.float64)).T) + 2 * u * np.abs(lref)
     if bias is not None:
         bound += u * np.abs(bias)
-    assert (np.abs(logits.cpu().numpy() - lref) <= bound).all()
+    lg = logits.cpu().numpy().astype(np.float64)
+    assert (np.abs(lg - lref) <= bound).all()
+    # every token: the indices are the top-k of the GPU's own float32 logits
+    # (ties to the lower index), the weights their renormalised softmax
+    fi, fw = O.route_topk(lg, cfg.k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), fi)
+    np.testing.assert_allclose(w.cpu().numpy(), fw, atol=TOL_W, rtol=0)
     ref = {"logits": lref, "idx": iref, "w": wref}
     L = {"x": x, "W_r": W_r, "bias": bias}
-    check_routing(L, ref, idx.cpu().numpy(), w.cpu().numpy(), cfg.k, cfg.H)
+    # near-ties (fp64 gaps under the float32 bound) are a few percent of the
+    # tokens of the 300-token batch (k adjacent gaps per token, each must
+    # clear about 1e-3 there) and none of the decode batches
+    check_routing(L, ref, idx.cpu().numpy(), w.cpu().numpy(), cfg.k, cfg.H,
+                  max_ties=0 if T <= 37 else T // 10)
 
 
 @pytest.mark.parametrize("T,E,k", [(1, 8, 2), (5, 64, 2), (37, 256, 8), (4096, 256, 8),
@@ -197,10 +207,7 @@ def test_layer_forward(name, T):
     ref = O.layer_forward(L["x"], L["W_r"], L["bias"], L["experts"], L["shared"], cfg.k)
     out = gpu_layer(L, dev_layer(L), cfg)
     check_routing(L, ref, out["idx"], out["w"], cfg.k, cfg.H)
-    want = O.bf16_bits_to_f64(ref["y_bf16"])
-    got = O.bf16_bits_to_f64(out["y"])
-    assert rel_l2(got, want) < TOL_Y
-    assert rel_l2(got, ref["y"]) < TOL_Y
+    check_y(out["y"], ref)
 
 
 def test_layer_forward_mxfp4_act_mode():
@@ -208,7 +215,7 @@ def test_layer_forward_mxfp4_act_mode():
     L = synth.layer(cfg, 2, 16)
     ref = O.layer_forward(L["x"], L["W_r"], L["bias"], L["experts"], L["shared"], cfg.k, "mxfp4_act")
     out = gpu_layer(L, dev_layer(L), cfg, moe.MOE_PATH_GEMV, moe.MOE_ACT_MXFP4)
-    assert rel_l2(O.bf16_bits_to_f64(out["y"]), O.bf16_bits_to_f64(ref["y_bf16"])) < TOL_Y
+    check_y(out["y"], ref)
 
 
 EDGE = [
@@ -229,25 +236,22 @@ def test_layer_edge_shapes(H, I, E, k, T, shared, bias):
     ref = O.layer_forward(L["x"], L["W_r"], L["bias"], L["experts"], L["shared"], k)
     out = gpu_layer(L, dev_layer(L), cfg)
     check_routing(L, ref, out["idx"], out["w"], k, H)
-    assert rel_l2(O.bf16_bits_to_f64(out["y"]), O.bf16_bits_to_f64(ref["y_bf16"])) < TOL_Y
+    check_y(out["y"], ref)
 
 
-def test_h_beyond_f16_range_latches_device_data():
+def test_h_beyond_f16_range_is_carried_exactly():
     """The row-block GEMV carries the SwiGLU output to the down projection as
-    an f16 pair: an |h| that f16 cannot hold must latch an error, not turn
-    into infinities.  Every weight 6 * 2^13 and x = 1 give |g|, |u| ~ 1.3e7."""
+    an f16 pair with a power of two per 32 values, so an |h| far beyond the
+    f16 range is still exact.  Every weight 6 * 2^13 and x = 1 give |g|, |u|
+    ~ 1.3e7 and h ~ 1.6e14."""
     cfg = synth.TINY
     L = synth.layer(cfg, 0)
     L["experts"] = {n: (np.full_like(a, 0x77) if n.endswith("_q") else np.full_like(a, 140))
                     for n, a in L["experts"].items()}
     L["x"] = np.full_like(L["x"], 0x3F80)   # bf16 1.0
-    D = dev_layer(L)
-    shape = moe.shape_of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k)
-    ws = moe.make_workspace(shape, moe.MOE_PATH_GEMV)
-    y = torch.empty((cfg.T, cfg.H), dtype=torch.int16, device="cuda")
-    moe.moe_layer_forward(D["x"], D["W_r"], None, D["experts"], None, shape, y, ws)
-    torch.cuda.synchronize()
-    assert moe.moe_get_error(ws) == moe.MOE_ERR_DEVICE_DATA
+    ref = O.layer_forward(L["x"], L["W_r"], None, L["experts"], None, cfg.k)
+    out = gpu_layer(L, dev_layer(L), cfg, moe.MOE_PATH_GEMV, moe.MOE_ACT_EXACT)
+    check_y(out["y"], ref)
 
 
 def test_one_hot_and_zero_experts():
@@ -259,11 +263,11 @@ def test_one_hot_and_zero_experts():
     ref = O.layer_forward(L["x"], L["W_r"], L["bias"], L["experts"], L["shared"], 1)
     out = gpu_layer(L, dev_layer(L), cfg)
     assert (out["idx"][:, 0] == 5).all() and (out["w"] == 1.0).all()
-    assert rel_l2(O.bf16_bits_to_f64(out["y"]), O.bf16_bits_to_f64(ref["y_bf16"])) < TOL_Y
+    check_y(out["y"], ref)
     L["experts"] = {n: np.zeros_like(a) for n, a in L["experts"].items()}
     ref = O.layer_forward(L["x"], L["W_r"], L["bias"], L["experts"], L["shared"], 1)
     out = gpu_layer(L, dev_layer(L), cfg)
-    assert rel_l2(O.bf16_bits_to_f64(out["y"]), O.bf16_bits_to_f64(ref["y_bf16"])) < TOL_Y
+    check_y(out["y"], ref)
 
 
 def test_graph_replay_matches_eager():
@@ -286,7 +290,7 @@ def test_graph_replay_matches_eager():
     g.replay()
     torch.cuda.synchronize()
     ref = O.layer_forward(x2, L["W_r"], None, L["experts"], None, cfg.k)
-    assert rel_l2(O.bf16_bits_to_f64(bits_np(y)), O.bf16_bits_to_f64(ref["y_bf16"])) < TOL_Y
+    check_y(bits_np(y), ref)
     D["x"].copy_(to_dev_bits(L["x"]))
     g.replay()
     torch.cuda.synchronize()

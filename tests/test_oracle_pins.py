@@ -416,3 +416,38 @@ def test_near_tie_bound_flags_exact_ties_only_when_close():
     assert ties.tolist() == [0, 1]
     W2 = np.array([[1.0, 0, 0, 0], [0.5, 0, 0, 0], [0.25, 0, 0, 0]])
     assert O.near_tie_tokens(x, W2, None, O.router_logits(x, W2, None), 1, depth=8).size == 0
+
+
+def _tie_threshold(depth, la, sa, sb, ba, bb):
+    """Exact gap g at which logits la and la - g (with sum|x W| of sa and sb,
+    biases ba and bb) meet the bound: g (1 + 2u) = gamma (sa + sb)
+    + 4u la + u (|ba| + |bb|), u = 2^-24, gamma = depth u / (1 - depth u)."""
+    u = Fraction(1, 2 ** 24)
+    gamma = depth * u / (1 - depth * u)
+    return (gamma * (Fraction(sa) + Fraction(sb)) + 4 * u * Fraction(la)
+            + u * (abs(Fraction(ba)) + abs(Fraction(bb)))) / (1 + 2 * u)
+
+
+@pytest.mark.parametrize("depth", [8, 41])
+@pytest.mark.parametrize("bias", [None, (0.5, 0.25, 0.0)])
+def test_near_tie_bound_magnitude_exact(depth, bias):
+    """The near-tie bound is Higham's gamma_depth * sum|x W| plus 2u|logit|
+    (plus u|b|) per logit, u = 2^-24: a gap just below the exact bound (as a
+    rational) is a near-tie, one just above is not.  A wrong unit roundoff, a
+    dropped gamma or a scaled bound moves one of the two cases across."""
+    x = np.array([[1.0, 0.0, 0.0, 0.0]])
+    W = np.array([[1.0, 0, 0, 0], [-1.0, 0, 0, 0], [0.125, 0, 0, 0]])
+    b = None if bias is None else np.array(bias)
+    bz = (0.0, 0.0, 0.0) if bias is None else bias
+    eps = Fraction(1, 10 ** 6)
+    # k = 1: the top two logits 1 and 1 - g
+    g01 = _tie_threshold(depth, 1, 1, 1, bz[0], bz[1])
+    for scale, expect_tie in ((1 - eps, True), (1 + eps, False)):
+        logits = np.array([[1.0, 1.0 - float(g01 * scale), -10.0]])
+        assert (O.near_tie_tokens(x, W, b, logits, 1, depth).size == 1) == expect_tie
+    # k = 2: the order among the top k + 1 counts too; logits 1, 0.5 and
+    # 0.5 - g (experts 1 and 2: sum|x W| 1 and 0.125)
+    g12 = _tie_threshold(depth, 0.5, 1, 0.125, bz[1], bz[2])
+    for scale, expect_tie in ((1 - eps, True), (1 + eps, False)):
+        logits = np.array([[1.0, 0.5, 0.5 - float(g12 * scale)]])
+        assert (O.near_tie_tokens(x, W, b, logits, 2, depth).size == 1) == expect_tie
