@@ -43,6 +43,7 @@ constexpr int kBM = 128;            // weight rows per item (MMA M)
 constexpr int kBKB = 128;           // K bytes per stage (256 FP4 values)
 constexpr int kGemmThreads = 192;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
+constexpr int kSmallN = 16;         // token rows of the small activation box
 
 template <int PHASE>
 struct GemmCfg {
@@ -61,6 +62,7 @@ struct GemmCfg {
   static constexpr int BUDGET = 216 * 1024 - EPI_BYTES;
   static constexpr int NS = BUDGET / STAGE > 8 ? 8 : BUDGET / STAGE;
   static constexpr int SMEM = NS * STAGE + EPI_BYTES + 1024 /*barriers*/ + 1024 /*alignment*/;
+  // plus, after SMEM, the per-virtual-expert routing tables (tables_bytes)
   // TMEM columns: two accumulator buffers, then scale factors
   static constexpr int ACC_COLS = NPROJ * BN;
   static constexpr int SFA_COL = 2 * ACC_COLS;              // NPROJ * 8 columns
@@ -233,30 +235,35 @@ struct Item {
   int nvalid;   // tokens of this item
 };
 
+// Per-virtual-expert routing tables, staged in shared memory once per CTA:
+// items before v (nV + 1 entries), expert id (or -1), first activation row
+// and tokens of v.
+struct Tables {
+  const int* item_off;
+  const int* e;
+  const int* row0;
+  const int* R;
+};
+__host__ __device__ inline size_t tables_bytes(int E) { return size_t(4) * 4 * (E + 2); }
+
 template <int BN>
-__device__ __forceinline__ Item item_of(const GemmArgs& a, int it, int nA, int nV, int MT) {
+__device__ __forceinline__ Item item_of(const Tables& tb, int it, int nV, int MT) {
   // virtual expert: last v with item_off[v] <= it
   int lo = 0, hi = nV - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (a.item_off[mid] <= it) lo = mid;
+    if (tb.item_off[mid] <= it) lo = mid;
     else hi = mid - 1;
   }
   Item r;
   r.v = lo;
-  const int li = it - a.item_off[lo];
-  const int ntiles = (a.item_off[lo + 1] - a.item_off[lo]) / MT;
+  const int li = it - tb.item_off[lo];
+  const int ntiles = (tb.item_off[lo + 1] - tb.item_off[lo]) / MT;
   r.mt = li / ntiles;
   r.nt = li % ntiles;  // token tiles fastest: neighbours share the weight tile in L2
-  if (lo < nA) {
-    r.e = a.plan[1 + lo];
-    r.row0 = a.offsets[r.e];
-    r.R = a.offsets[r.e + 1] - r.row0;
-  } else {
-    r.e = -1;
-    r.row0 = a.T * a.k;
-    r.R = a.T;
-  }
+  r.e = tb.e[lo];
+  r.row0 = tb.row0[lo];
+  r.R = tb.R[lo];
   r.nvalid = min(BN, r.R - r.nt * BN);
   return r;
 }
@@ -266,7 +273,8 @@ template <int PHASE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     k_ffn_gemm(GemmArgs a, const __grid_constant__ CUtensorMap mA0,
                const __grid_constant__ CUtensorMap mA1, const __grid_constant__ CUtensorMap mS0,
-               const __grid_constant__ CUtensorMap mS1, const __grid_constant__ CUtensorMap mB) {
+               const __grid_constant__ CUtensorMap mS1, const __grid_constant__ CUtensorMap mB,
+               const __grid_constant__ CUtensorMap mBs) {
   using C = GemmCfg<PHASE>;
   constexpr int NPROJ = C::NPROJ;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -281,6 +289,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_tab = reinterpret_cast<int*>(smem + C::SMEM - 1024);  // after the barriers' kilobyte
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -307,9 +316,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) {
+    // the descriptors are fetched while the previous kernel drains
+    const void* maps[6] = {&mA0, &mA1, &mS0, &mS1, &mB, &mBs};
+#pragma unroll
+    for (int i = 0; i < 6; ++i) asm volatile("prefetch.tensormap [%0];" ::"l"(maps[i]) : "memory");
+  }
 
   pdl_wait();
   pdl_trigger();
+
+  // routing tables -> shared memory (one round of loads)
+  Tables tb;
+  {
+    const int nA0 = __ldg(a.plan);
+    const int nV0 = nA0 + (a.has_shared ? 1 : 0);
+    int* t_off = s_tab;
+    int* t_e = t_off + (a.E + 2);
+    int* t_row0 = t_e + (a.E + 2);
+    int* t_R = t_row0 + (a.E + 2);
+    for (int v = threadIdx.x; v <= nV0; v += blockDim.x) {
+      t_off[v] = __ldg(a.item_off + v);
+      if (v < nA0) {
+        const int e = __ldg(a.plan + 1 + v);
+        const int r0 = __ldg(a.offsets + e);
+        t_e[v] = e;
+        t_row0[v] = r0;
+        t_R[v] = __ldg(a.offsets + e + 1) - r0;
+      } else if (v < nV0) {
+        t_e[v] = -1;
+        t_row0[v] = a.T * a.k;
+        t_R[v] = a.T;
+      }
+    }
+    __syncthreads();
+    tb.item_off = t_off;
+    tb.e = t_e;
+    tb.row0 = t_row0;
+    tb.R = t_R;
+  }
 
   const int K = PHASE == 0 ? a.H : a.I;
   const int ROWS = PHASE == 0 ? a.I : a.H;
@@ -317,13 +362,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int NSC = K / 32;      // scale bytes per row
   const int nks = (KB + kBKB - 1) / kBKB;
   const int MT = ROWS / kBM;
-  const int nA = a.plan[0];
+  const int nA = __ldg(a.plan);
   const int nV = nA + (a.has_shared ? 1 : 0);
-  const int n_items = a.item_off[nV];
+  const int n_items = tb.item_off[nV];
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // Stages are numbered g = 0.. over this CTA's items (nks stages each).
+    // Items of at most kSmallN tokens load a kSmallN-row activation box
+    // instead of BN rows.
     // The scale words of stage g+1 are loaded into registers while stage g
     // waits for its slot, so their global latency overlaps the pipeline; the
     // tile TMAs are issued before the scales are written, and the stage's full
@@ -342,7 +389,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     auto prepare = [&](int g) {
       ks_n = g % nks;
       if (ks_n == 0) {
-        wn = item_of<C::BN>(a, int(blockIdx.x) + (g / nks) * int(gridDim.x), nA, nV, MT);
+        wn = item_of<C::BN>(tb, int(blockIdx.x) + (g / nks) * int(gridDim.x), nV, MT);
         arow_n = (wn.e >= 0 ? wn.e * ROWS : 0) + wn.mt * kBM;
         brow_n = wn.row0 + wn.nt * C::BN;
       }
@@ -378,6 +425,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int g = 0; g < total && ok; ++g) {
       const int ks = ks_n, arow = arow_n, brow = brow_n;
       const bool routed = wn.e >= 0;
+      const bool small = wn.nvalid <= kSmallN;
       uint32_t sa[NPROJ][4][2], sb[NB_ROWS][2];
 #pragma unroll
       for (int p = 0; p < NPROJ; ++p)
@@ -403,11 +451,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (lane == 0) {
         uint64_t pol;
         asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-        mbar_expect_tx(fb, NPROJ * C::A_BYTES + C::B_BYTES);
+        mbar_expect_tx(fb, NPROJ * C::A_BYTES + (small ? kSmallN : C::BN) * kBKB);
         tma_load_2d_hint(saddr(st), routed ? &mA0 : &mS0, ks * kBKB, arow, fb, pol);
         if constexpr (NPROJ == 2)
           tma_load_2d_hint(saddr(st + C::A_BYTES), routed ? &mA1 : &mS1, ks * kBKB, arow, fb, pol);
-        tma_load_2d(saddr(st + NPROJ * C::A_BYTES), &mB, ks * kBKB, brow, fb);
+        tma_load_2d(saddr(st + NPROJ * C::A_BYTES), small ? &mBs : &mB, ks * kBKB, brow, fb);
       }
       // scale words -> atom layout: K atom `at` of row r at at*512 + 16*(r%32) + 4*(r/32%4)
 #pragma unroll
@@ -454,7 +502,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t tsfb = tmem + C::SFB_COL;
       int local = 0;  // items of this CTA so far: buffer local & 1, use local >> 1
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++local) {
-        const Item w = item_of<C::BN>(a, it, nA, nV, MT);
+        const Item w = item_of<C::BN>(tb, it, nV, MT);
         const int n_mma = ((w.nvalid + 7) / 8) * 8;
         const int buf = local & 1;
         const uint32_t acc_parity = (uint32_t(local >> 1) & 1u) ^ 1u;
@@ -516,7 +564,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     float* tile = epi + q * 32 * 33;  // 32 x 32 transpose tile (phase 0)
     int local = 0;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++local) {
-      const Item w = item_of<C::BN>(a, it, nA, nV, MT);
+      const Item w = item_of<C::BN>(tb, it, nV, MT);
       const int buf = local & 1;
       if (!warp_wait(saddr(&acc_full[buf]), uint32_t(local >> 1) & 1u, abort_flag, a.err, 300))
         break;
@@ -721,13 +769,14 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t row
 template <int PHASE>
 cudaError_t launch_gemm_phase(const GemmArgs& g, const CUtensorMap& a0, const CUtensorMap& a1,
                               const CUtensorMap& s0, const CUtensorMap& s1, const CUtensorMap& b,
-                              cudaStream_t st) {
+                              const CUtensorMap& bs, cudaStream_t st) {
   using C = GemmCfg<PHASE>;
   auto kern = k_ffn_gemm<PHASE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  const size_t smem = size_t(C::SMEM) + tables_bytes(g.E);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(device_info().sm_count), dim3(kGemmThreads), size_t(C::SMEM), st, g,
-                    a0, a1, s0, s1, b);
+  return launch_pdl(kern, dim3(device_info().sm_count), dim3(kGemmThreads), smem, st, g, a0, a1, s0,
+                    s1, b, bs);
 }
 
 }  // namespace
@@ -765,7 +814,11 @@ bool make_tma_map_u8_plain(CUtensorMap* m, const void* base, uint64_t row_bytes,
 }
 
 bool gemm_supported(const moe_shape_t& s) {
-  return s.H % 256 == 0 && s.I % 128 == 0 && encode_fn() != nullptr;
+  // the routing tables of E experts share the opt-in shared memory (227 KB)
+  // with the pipeline stages
+  const size_t cap = 227 * 1024, tab = tables_bytes(s.E);
+  return s.H % 256 == 0 && s.I % 128 == 0 && size_t(GemmCfg<0>::SMEM) + tab <= cap &&
+         size_t(GemmCfg<1>::SMEM) + tab <= cap && encode_fn() != nullptr;
 }
 
 cudaError_t launch_ffn_gemm(const FfnArgs& a, const GemmBuffers& gb, cudaStream_t st) {
@@ -777,13 +830,15 @@ cudaError_t launch_ffn_gemm(const FfnArgs& a, const GemmBuffers& gb, cudaStream_
                  a.has_shared, a.I / kBM, a.H / kBM, gb.item_off0, gb.item_off1);
   if (e != cudaSuccess) return e;
 
-  CUtensorMap g0, g1, sg0, sg1, bx, d0, sd0, bh;
+  CUtensorMap g0, g1, sg0, sg1, bx, bxs, d0, sd0, bh, bhs;
   const uint64_t HB = a.H / 2, IB = a.I / 2;
   bool ok = make_map(&g0, a.ex.gq, HB, uint64_t(a.E) * a.I, kBM) &&
             make_map(&g1, a.ex.uq, HB, uint64_t(a.E) * a.I, kBM) &&
             make_map(&bx, gb.xq, HB, rows, GemmCfg<0>::BN) &&
+            make_map(&bxs, gb.xq, HB, rows, kSmallN) &&
             make_map(&d0, a.ex.dq, IB, uint64_t(a.E) * a.H, kBM) &&
-            make_map(&bh, gb.hq, IB, rows, GemmCfg<1>::BN);
+            make_map(&bh, gb.hq, IB, rows, GemmCfg<1>::BN) &&
+            make_map(&bhs, gb.hq, IB, rows, kSmallN);
   if (a.has_shared) {
     ok = ok && make_map(&sg0, a.sh.gq, HB, a.I, kBM) && make_map(&sg1, a.sh.uq, HB, a.I, kBM) &&
          make_map(&sd0, a.sh.dq, IB, a.H, kBM);
@@ -814,7 +869,7 @@ cudaError_t launch_ffn_gemm(const FfnArgs& a, const GemmBuffers& gb, cudaStream_
   g.sb = gb.xs;
   g.hq = gb.hq;
   g.hs = gb.hs;
-  e = launch_gemm_phase<0>(g, g0, g1, sg0, sg1, bx, st);
+  e = launch_gemm_phase<0>(g, g0, g1, sg0, sg1, bx, bxs, st);
   if (e != cudaSuccess) return e;
   // phase 1: down
   g.item_off = gb.item_off1;
@@ -824,7 +879,7 @@ cudaError_t launch_ffn_gemm(const FfnArgs& a, const GemmBuffers& gb, cudaStream_
   g.sa_sh[1] = g.sa_sh[0];
   g.sb = gb.hs;
   g.partial = a.partial;
-  return launch_gemm_phase<1>(g, d0, d0, sd0, sd0, bh, st);
+  return launch_gemm_phase<1>(g, d0, d0, sd0, sd0, bh, bhs, st);
 }
 
 }  // namespace moe
