@@ -145,7 +145,7 @@ typedef struct moe_mxfp4_experts {
 
 /* Bytes of workspace the calls below need for this shape (any of them).
  * has_shared: 1 if a shared expert is passed.  Returns 0 for an unsupported
- * shape, path or precision. */
+ * shape, path or precision (k may exceed E, as for moe_expert_ffn_mxfp4). */
 MOE_API size_t moe_workspace_bytes(moe_shape_t shape, int32_t path, int32_t precision,
                            int32_t has_shared);
 
@@ -183,7 +183,9 @@ MOE_API moe_status_t moe_bucket(const int32_t* topk_idx, moe_shape_t shape,
  *   partial[T*k+t]  = the same through the shared expert.
  * `experts` and `shared` are host pointers to structs of device pointers;
  * experts->n_experts must equal shape.E, shared->n_experts must be 1.
- * Rows of pairs not listed in entries are left untouched. */
+ * Rows of pairs not listed in entries are left untouched.  Here k only sets
+ * the pair layout and may exceed shape.E (a rank holding a share of the
+ * experts, with offsets pointing at its experts' bucket starts). */
 MOE_API moe_status_t moe_expert_ffn_mxfp4(const moe_mxfp4_experts_t* experts,
                                   const moe_mxfp4_experts_t* shared,
                                   const uint16_t* x, const int32_t* offsets,
@@ -198,6 +200,22 @@ MOE_API moe_status_t moe_expert_ffn_mxfp4(const moe_mxfp4_experts_t* experts,
 MOE_API moe_status_t moe_combine(const float* partial, const float* topk_w,
                          moe_shape_t shape, int32_t has_shared, uint16_t* y,
                          void* stream);
+
+/* Expert-parallel pieces (a group of ranks each holding a contiguous range of
+ * the routed experts; the pages run on one device, this spreads the same
+ * layer over several):
+ *   y_f32[t] = sum over j < k with e_begin <= topk_idx[t,j] < e_end of
+ *              topk_w[t,j] * partial[t*k+j]  (+ partial[T*k+t] if has_shared),
+ * summed in slot order in float32 and left in float32 [T, H] so the ranks'
+ * results can be added (one all-reduce); rows of pairs outside the range are
+ * not read.  0 <= e_begin <= e_end <= shape.E. */
+MOE_API moe_status_t moe_combine_range(const float* partial, const float* topk_w,
+                                       const int32_t* topk_idx, int32_t e_begin, int32_t e_end,
+                                       moe_shape_t shape, int32_t has_shared, float* y_f32,
+                                       void* stream);
+
+/* out[i] = bf16_rne(in[i]) for n float32 values (n % 4 == 0). */
+MOE_API moe_status_t moe_round_bf16(const float* in, int64_t n, uint16_t* out, void* stream);
 
 /* The whole layer: route -> bucket -> expert FFNs -> combine, on `stream`.
  * topk_idx_out [T,k] and topk_w_out [T,k] may be NULL (kept in ws then). */

@@ -45,6 +45,15 @@ moe_status_t check_shape(const moe_shape_t& s) {
   return MOE_OK;
 }
 
+// The expert-FFN entry: k only describes the pair layout (p = t*k + j), so it
+// may exceed the number of experts passed (one rank's share of them).
+moe_status_t check_ffn_shape(const moe_shape_t& s) {
+  moe_shape_t r = s;
+  r.k = 1;
+  if (check_shape(r) != MOE_OK || s.k < 1 || s.k > kMaxTopK) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
 moe_status_t check_ptrs(std::initializer_list<const void*> required) {
   for (const void* p : required)
     if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
@@ -134,7 +143,7 @@ extern "C" {
 
 size_t moe_workspace_bytes(moe_shape_t shape, int32_t path, int32_t precision,
                            int32_t has_shared) {
-  if (check_shape(shape) != MOE_OK || !valid_path(path) || !valid_precision(precision)) return 0;
+  if (check_ffn_shape(shape) != MOE_OK || !valid_path(path) || !valid_precision(precision)) return 0;
   const int gemm = path != MOE_PATH_GEMV;
   return ws_layout(shape, has_shared != 0, gemm).total;
 }
@@ -207,7 +216,7 @@ moe_status_t moe_expert_ffn_mxfp4(const moe_mxfp4_experts_t* experts,
                                   const int32_t* offsets, const int32_t* entries,
                                   moe_shape_t shape, int32_t path, int32_t precision,
                                   float* partial_out, void* ws, size_t ws_bytes, void* stream) {
-  moe_status_t st = check_shape(shape);
+  moe_status_t st = check_ffn_shape(shape);
   if (st != MOE_OK) return st;
   if (!valid_path(path) || !valid_precision(precision)) return MOE_ERR_INVALID_ARG;
   st = check_experts(experts, shape.E);
@@ -267,6 +276,27 @@ moe_status_t moe_combine(const float* partial, const float* topk_w, moe_shape_t 
   if (st != MOE_OK) return st;
   return cuda_status(launch_combine(partial, topk_w, shape.T, shape.H, shape.k, has_shared != 0,
                                     y, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_combine_range(const float* partial, const float* topk_w, const int32_t* topk_idx,
+                               int32_t e_begin, int32_t e_end, moe_shape_t shape,
+                               int32_t has_shared, float* y_f32, void* stream) {
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  st = check_ptrs({partial, topk_w, topk_idx, y_f32});
+  if (st != MOE_OK) return st;
+  if (e_begin < 0 || e_end < e_begin || e_end > shape.E) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_combine_range(partial, topk_w, topk_idx, e_begin, e_end, shape.T,
+                                          shape.H, shape.k, has_shared != 0, y_f32,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_round_bf16(const float* in, int64_t n, uint16_t* out, void* stream) {
+  if (n < 0 || n % 4) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (n == 0) return MOE_OK;
+  moe_status_t st = check_ptrs({in, out});
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_round_bf16(in, n, out, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router, const float* bias,

@@ -497,6 +497,55 @@ __global__ void __launch_bounds__(256) k_combine(const float* partial, const flo
   *reinterpret_cast<uint2*>(y + size_t(t) * H + c) = out;
 }
 
+// Float32 combine of the pairs whose expert lies in [e_begin, e_end) (the
+// experts one rank of an expert-parallel group holds): the same slot-order
+// sums as k_combine, left in float32 for a sum over ranks.
+__global__ void __launch_bounds__(256) k_combine_range(const float* partial, const float* w,
+                                                       const int32_t* idx, int e_begin, int e_end,
+                                                       int T, int H, int k, int has_shared,
+                                                       float* y) {
+  pdl_wait();
+  pdl_trigger();
+  const int per_row = H / 4;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)T * per_row) return;
+  const int t = int(i / per_row), c = int(i % per_row) * 4;
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < k; ++j) {
+    const int e = __ldg(idx + size_t(t) * k + j);
+    if (e < e_begin || e >= e_end) continue;
+    const float wj = __ldg(w + size_t(t) * k + j);
+    const float4 p = __ldcg(reinterpret_cast<const float4*>(partial + (size_t(t) * k + j) * H + c));
+    s.x = fmaf(wj, p.x, s.x);
+    s.y = fmaf(wj, p.y, s.y);
+    s.z = fmaf(wj, p.z, s.z);
+    s.w = fmaf(wj, p.w, s.w);
+  }
+  if (has_shared) {
+    const float4 p =
+        __ldcg(reinterpret_cast<const float4*>(partial + (size_t(T) * k + t) * H + c));
+    s.x += p.x;
+    s.y += p.y;
+    s.z += p.z;
+    s.w += p.w;
+  }
+  *reinterpret_cast<float4*>(y + size_t(t) * H + c) = s;
+}
+
+// float32 -> bf16 (round to nearest even), four values per thread.
+__global__ void __launch_bounds__(256) k_round_bf16(const float* in, long long n4, uint16_t* out) {
+  pdl_wait();
+  pdl_trigger();
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const float4 v = __ldcg(reinterpret_cast<const float4*>(in) + i);
+  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+  uint2 o;
+  o.x = *reinterpret_cast<uint32_t*>(&lo);
+  o.y = *reinterpret_cast<uint32_t*>(&hi);
+  reinterpret_cast<uint2*>(out)[i] = o;
+}
+
 // bf16 token rows -> scaled f16 rows and their exponents (for calls that do
 // not route through the fused router): one warp per token row finds the
 // row's largest magnitude, then converts its 32-value blocks.  The grid also
@@ -561,6 +610,21 @@ cudaError_t launch_combine(const float* partial, const float* w, int T, int H, i
   const int blocks = int((n + 255) / 256);
   return launch_pdl(k_combine, dim3(blocks), dim3(256), 0, st, partial, w, T, H, k, has_shared,
                     y);
+}
+
+cudaError_t launch_combine_range(const float* partial, const float* w, const int32_t* idx,
+                                 int e_begin, int e_end, int T, int H, int k, int has_shared,
+                                 float* y, cudaStream_t st) {
+  const long long n = (long long)T * (H / 4);
+  const int blocks = int((n + 255) / 256);
+  return launch_pdl(k_combine_range, dim3(blocks), dim3(256), 0, st, partial, w, idx, e_begin, e_end,
+                    T, H, k, has_shared, y);
+}
+
+cudaError_t launch_round_bf16(const float* in, long long n, uint16_t* out, cudaStream_t st) {
+  const long long n4 = n / 4;
+  if (n4 == 0) return cudaSuccess;
+  return launch_pdl(k_round_bf16, dim3(unsigned((n4 + 255) / 256)), dim3(256), 0, st, in, n4, out);
 }
 
 }  // namespace moe

@@ -444,6 +444,10 @@ bool gemm_supported(const moe_shape_t& s);
 cudaError_t launch_ffn_gemm(const FfnArgs& a, const GemmBuffers& gb, cudaStream_t st);
 cudaError_t launch_combine(const float* partial, const float* w, int T, int H, int k,
                            int has_shared, uint16_t* y, cudaStream_t st);
+cudaError_t launch_combine_range(const float* partial, const float* w, const int32_t* idx,
+                                 int e_begin, int e_end, int T, int H, int k, int has_shared,
+                                 float* y, cudaStream_t st);
+cudaError_t launch_round_bf16(const float* in, long long n, uint16_t* out, cudaStream_t st);
 cudaError_t launch_act_quant(const float* in, int rows, int K, uint8_t* q, uint8_t* s,
                              cudaStream_t st);
 // words[0] = w0, words[1] = w1 (one thread; ordered on the stream).

@@ -40,6 +40,7 @@ EXPORTS = (
     "moe_expert_ffn_mxfp4", "moe_combine", "moe_layer_forward", "moe_act_quant_mxfp4",
     "moe_decode_mxfp4", "moe_get_error", "moe_status_string", "moe_version",
     "moe_layer_forward_static", "moe_get_error_static", "moe_workspace_set_limits",
+    "moe_combine_range", "moe_round_bf16",
 )
 
 
@@ -85,6 +86,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "moe_bucket": (i32, [vp, shape, vp, vp, vp, vp, sz, vp]),
         "moe_expert_ffn_mxfp4": (i32, [ex, ex, vp, vp, vp, shape, i32, i32, vp, vp, sz, vp]),
         "moe_combine": (i32, [vp, vp, shape, i32, vp, vp]),
+        "moe_combine_range": (i32, [vp, vp, vp, i32, i32, shape, i32, vp, vp]),
+        "moe_round_bf16": (i32, [vp, ctypes.c_int64, vp, vp]),
         "moe_layer_forward": (i32, [vp, vp, vp, ex, ex, shape, i32, i32, vp, vp, vp, vp, sz, vp]),
         "moe_layer_forward_static": (i32, [vp, vp, vp, ex, ex, shape, i32, vp, vp, vp, vp]),
         "moe_act_quant_mxfp4": (i32, [vp, i32, i32, vp, vp, vp]),
@@ -212,6 +215,18 @@ def moe_expert_ffn_mxfp4(experts: Experts, shared, x, offsets, entries, shape, p
 def moe_combine(partial, topk_w, shape, has_shared, y, stream=None):
     _check(load_library().moe_combine(_p(partial), _p(topk_w), shape, int(has_shared), _p(y),
                                       _s(stream)), "moe_combine")
+
+
+def moe_combine_range(partial, topk_w, topk_idx, e_begin, e_end, shape, has_shared, y_f32,
+                      stream=None):
+    _check(load_library().moe_combine_range(_p(partial), _p(topk_w), _p(topk_idx), e_begin, e_end,
+                                            shape, int(has_shared), _p(y_f32), _s(stream)),
+           "moe_combine_range")
+
+
+def moe_round_bf16(x_f32, out, stream=None):
+    _check(load_library().moe_round_bf16(_p(x_f32), x_f32.numel(), _p(out), _s(stream)),
+           "moe_round_bf16")
 
 
 def moe_layer_forward(x, w_router, bias, experts: Experts, shared, shape, y, ws,

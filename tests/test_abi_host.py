@@ -46,7 +46,7 @@ def test_workspace_bytes():
     assert moe.moe_workspace_bytes(s, moe.MOE_PATH_GEMV, has_shared=True) > n_gemv
     assert moe.moe_workspace_bytes(s, moe.MOE_PATH_AUTO) >= n_gemv
     for bad in [(0, 4096, 1408, 64, 2), (1, 4016, 1408, 64, 2), (1, 4096, 1400, 64, 2),
-                (1, 4096, 1408, 2000, 2), (1, 4096, 1408, 8, 9), (1, 4096, 1408, 64, 17)]:
+                (1, 4096, 1408, 2000, 2), (1, 4096, 1408, 64, 17)]:
         assert moe.moe_workspace_bytes(moe.shape_of(*bad)) == 0, bad
     assert moe.moe_workspace_bytes(s, path=7) == 0
     assert moe.moe_workspace_bytes(s, precision=3) == 0
@@ -93,3 +93,16 @@ def test_rejects_bad_arguments_before_launch(lib):
     assert lib.moe_decode_mxfp4(_fake(A), None, 4, 64, _fake(A), None) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_get_error(None, None) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_workspace_init(_fake(A + 8), 1024, None) == moe.MOE_ERR_INVALID_ARG
+    # routing needs k <= E; the expert FFN only needs k <= 16 (pair layout)
+    k_gt_e = moe.shape_of(4, 256, 128, 4, 8)
+    assert lib.moe_route_topk(_fake(A), _fake(A), None, k_gt_e, None, _fake(A), _fake(A), _fake(A),
+                              1 << 30, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert moe.moe_workspace_bytes(k_gt_e, moe.MOE_PATH_GEMV) > 0
+    assert moe.moe_workspace_bytes(moe.shape_of(4, 256, 128, 4, 17), moe.MOE_PATH_GEMV) == 0
+    # expert-parallel pieces
+    assert lib.moe_combine_range(_fake(A), _fake(A), _fake(A), 2, 9, s, 0, _fake(A),
+                                 None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine_range(_fake(A), _fake(A), None, 0, 8, s, 0, _fake(A),
+                                 None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_round_bf16(_fake(A), 6, _fake(A), None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert lib.moe_round_bf16(_fake(A), 0, _fake(A), None) == moe.MOE_OK
