@@ -259,6 +259,65 @@ MOE_API moe_status_t moe_layer_forward_static(const uint16_t* x, const float* w_
  * nothing. */
 MOE_API moe_status_t moe_get_error_static(void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Slot bank: the routed experts in pinned host memory, a bounded set of them
+ * resident in device memory.  The ds4-ssd engine streams the experts its
+ * router picks into a fixed expert cache ("ds4-ssd" README, "Run SSD Sidecar
+ * Mode"); here the backing store is pinned host memory and the bank a
+ * caller-owned device region of n_slots experts, filled least recently used
+ * first.  A bank is used from one host thread at a time.
+ * ------------------------------------------------------------------------- */
+typedef struct moe_slot_bank moe_slot_bank_t;
+
+/* Device bytes of a bank of n_slots experts of shape (H, I); 0 if invalid. */
+MOE_API size_t moe_slot_bank_bytes(int32_t H, int32_t I, int32_t n_slots);
+
+/* Create a bank over host_experts (HOST pointers to pinned memory, in the
+ * canonical layout, n_experts = E) with n_slots slots in slot_mem (device,
+ * 16-byte aligned, at least moe_slot_bank_bytes bytes, owned by the caller).
+ * The bank object and two small pinned host buffers (the call's expert ids,
+ * the expert -> slot map) are host memory the library allocates;
+ * moe_slot_bank_destroy frees them.  No device memory is allocated. */
+MOE_API moe_status_t moe_slot_bank_create(const moe_mxfp4_experts_t* host_experts, int32_t H,
+                                          int32_t I, int32_t n_slots, void* slot_mem,
+                                          size_t slot_mem_bytes, moe_slot_bank_t** out);
+MOE_API void moe_slot_bank_destroy(moe_slot_bank_t* bank);
+
+/* Make the experts ids[0..n) (host array) resident: experts already in the
+ * bank keep their slot, missing ones take the least recently used slots this
+ * call does not need, copied host -> device on `stream` (asynchronous);
+ * slot_of[i] (host) receives the slot of ids[i].  Calling it ahead of a layer
+ * call with the experts expected next prefetches them.  More distinct experts
+ * than slots returns MOE_ERR_WORKSPACE. */
+MOE_API moe_status_t moe_slot_bank_acquire(moe_slot_bank_t* bank, const int32_t* ids, int32_t n,
+                                           int32_t* slot_of, void* stream);
+
+/* The device experts struct of the bank's slots (n_experts = n_slots). */
+MOE_API moe_status_t moe_slot_bank_experts(const moe_slot_bank_t* bank,
+                                           moe_mxfp4_experts_t* out);
+
+/* Slot hits, misses (host -> device copies) and evictions so far. */
+MOE_API moe_status_t moe_slot_bank_stats(const moe_slot_bank_t* bank, int64_t* hits,
+                                         int64_t* misses, int64_t* evictions);
+
+/* The layer with its routed experts in a slot bank: route and top-k over all
+ * E experts on `stream`, the chosen experts read back to the host (this call
+ * synchronises the stream once), made resident, the indices rewritten to
+ * slots, then bucket, expert FFNs and combine over the bank.  Same inputs and
+ * output as moe_layer_forward; topk_idx_out / topk_w_out are required (expert
+ * ids and weights); T * k <= 8192; ws of at least
+ * moe_layer_forward_banked_workspace_bytes bytes. */
+MOE_API moe_status_t moe_layer_forward_banked(const uint16_t* x, const float* w_router,
+                                              const float* bias, moe_slot_bank_t* bank,
+                                              const moe_mxfp4_experts_t* shared,
+                                              moe_shape_t shape, int32_t path, int32_t precision,
+                                              uint16_t* y, int32_t* topk_idx_out,
+                                              float* topk_w_out, void* ws, size_t ws_bytes,
+                                              void* stream);
+MOE_API size_t moe_layer_forward_banked_workspace_bytes(moe_shape_t shape, int32_t n_slots,
+                                                        int32_t path, int32_t precision,
+                                                        int32_t has_shared);
+
 /* Quantise rows [rows, K] float32 to MXFP4 (codes [rows, K/2], scales
  * [rows, K/32]) with the MOE_ACT_MXFP4 rule above; K % 32 == 0. */
 MOE_API moe_status_t moe_act_quant_mxfp4(const float* in, int32_t rows, int32_t K,

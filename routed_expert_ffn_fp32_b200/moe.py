@@ -41,6 +41,9 @@ EXPORTS = (
     "moe_decode_mxfp4", "moe_get_error", "moe_status_string", "moe_version",
     "moe_layer_forward_static", "moe_get_error_static", "moe_workspace_set_limits",
     "moe_combine_range", "moe_round_bf16",
+    "moe_slot_bank_bytes", "moe_slot_bank_create", "moe_slot_bank_destroy", "moe_slot_bank_acquire",
+    "moe_slot_bank_experts", "moe_slot_bank_stats", "moe_layer_forward_banked",
+    "moe_layer_forward_banked_workspace_bytes",
 )
 
 
@@ -88,6 +91,15 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "moe_combine": (i32, [vp, vp, shape, i32, vp, vp]),
         "moe_combine_range": (i32, [vp, vp, vp, i32, i32, shape, i32, vp, vp]),
         "moe_round_bf16": (i32, [vp, ctypes.c_int64, vp, vp]),
+        "moe_slot_bank_bytes": (sz, [i32, i32, i32]),
+        "moe_slot_bank_create": (i32, [ex, i32, i32, i32, vp, sz, ctypes.POINTER(vp)]),
+        "moe_slot_bank_destroy": (None, [vp]),
+        "moe_slot_bank_acquire": (i32, [vp, vp, i32, vp, vp]),
+        "moe_slot_bank_experts": (i32, [vp, ex]),
+        "moe_slot_bank_stats": (i32, [vp, ctypes.POINTER(ctypes.c_int64),
+                                      ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64)]),
+        "moe_layer_forward_banked": (i32, [vp, vp, vp, vp, ex, shape, i32, i32, vp, vp, vp, vp, sz, vp]),
+        "moe_layer_forward_banked_workspace_bytes": (sz, [shape, i32, i32, i32, i32]),
         "moe_layer_forward": (i32, [vp, vp, vp, ex, ex, shape, i32, i32, vp, vp, vp, vp, sz, vp]),
         "moe_layer_forward_static": (i32, [vp, vp, vp, ex, ex, shape, i32, vp, vp, vp, vp]),
         "moe_act_quant_mxfp4": (i32, [vp, i32, i32, vp, vp, vp]),
@@ -227,6 +239,77 @@ def moe_combine_range(partial, topk_w, topk_idx, e_begin, e_end, shape, has_shar
 def moe_round_bf16(x_f32, out, stream=None):
     _check(load_library().moe_round_bf16(_p(x_f32), x_f32.numel(), _p(out), _s(stream)),
            "moe_round_bf16")
+
+
+class SlotBank:
+    """Routed experts in pinned host memory, n_slots of them resident in a
+    device slot bank (moe_slot_bank_*).  ``host`` holds CPU tensors in the
+    library's layout; they are pinned here if they are not already."""
+
+    def __init__(self, host: "Experts", H: int, I: int, n_slots: int, device="cuda"):
+        lib = load_library()
+        self.host = Experts(**{f: (t if t.is_pinned() else t.pin_memory())
+                               for f, t in dataclasses.asdict(host).items()})
+        n = int(lib.moe_slot_bank_bytes(H, I, n_slots))
+        if n == 0:
+            raise MoeError(MOE_ERR_UNSUPPORTED_SHAPE, "moe_slot_bank_bytes")
+        self.mem = torch.empty(n, dtype=torch.uint8, device=device)
+        self.n_slots = n_slots
+        h = self.host
+        hs = moe_mxfp4_experts_t(h.gate_q.data_ptr(), h.gate_s.data_ptr(), h.up_q.data_ptr(),
+                                 h.up_s.data_ptr(), h.down_q.data_ptr(), h.down_s.data_ptr(),
+                                 int(h.gate_q.shape[0]))
+        self._h = ctypes.c_void_p()
+        _check(lib.moe_slot_bank_create(ctypes.byref(hs), H, I, n_slots, self.mem.data_ptr(), n,
+                                        ctypes.byref(self._h)), "moe_slot_bank_create")
+
+    @property
+    def handle(self):
+        return self._h
+
+    def acquire(self, ids, stream=None):
+        """Make experts ``ids`` (ints) resident; returns their slots."""
+        arr = (ctypes.c_int32 * len(ids))(*ids)
+        out = (ctypes.c_int32 * len(ids))()
+        _check(load_library().moe_slot_bank_acquire(self._h, arr, len(ids), out, _s(stream)),
+               "moe_slot_bank_acquire")
+        return list(out)
+
+    def stats(self):
+        h, m, e = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        _check(load_library().moe_slot_bank_stats(self._h, ctypes.byref(h), ctypes.byref(m),
+                                                  ctypes.byref(e)), "moe_slot_bank_stats")
+        return h.value, m.value, e.value
+
+    def close(self):
+        if self._h:
+            load_library().moe_slot_bank_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def moe_layer_forward_banked(x, w_router, bias, bank: SlotBank, shared, shape, y, ws, topk_idx,
+                             topk_w, path=MOE_PATH_AUTO, precision=MOE_ACT_EXACT, stream=None):
+    _check(load_library().moe_layer_forward_banked(_p(x), _p(w_router), _p(bias), bank.handle,
+                                                   _ex(shared), shape, path, precision, _p(y),
+                                                   _p(topk_idx), _p(topk_w), _p(ws), ws.numel(),
+                                                   _s(stream)), "moe_layer_forward_banked")
+
+
+def banked_workspace(shape, n_slots, path=MOE_PATH_AUTO, precision=MOE_ACT_EXACT,
+                     has_shared=False, device="cuda", stream=None) -> torch.Tensor:
+    n = int(load_library().moe_layer_forward_banked_workspace_bytes(shape, n_slots, path, precision,
+                                                                    int(has_shared)))
+    if n == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED_SHAPE, "moe_layer_forward_banked_workspace_bytes")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    moe_workspace_init(ws, stream)
+    return ws
 
 
 def moe_layer_forward(x, w_router, bias, experts: Experts, shared, shape, y, ws,
