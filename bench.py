@@ -513,7 +513,54 @@ def run_extra(ls64, router64, args, stream, dev, peaks):
         ex[f"prefill_T{T}"] = entry(lsf, rp, pre, T, A, M, max(10, steps // 4), uses_tc=True)
     ex["sweep"] = sweep_rows(lsf, rp, synth.SWEEP, stream, reps=max(10, steps // 10),
                              variants=("gemv_mxfp4", "gemm_mxfp4"))
+    ex["banked_decode64_T5"] = banked_entry(ls64, router64, synth.DECODE64, 5, 32,
+                                            max(20, steps // 2), stream, dev)
     return ex
+
+
+def banked_entry(ls, router, cfg, T, n_slots, steps, stream, dev):
+    """The decode layer with its routed experts in pinned host memory and
+    n_slots of them in a device slot bank (least recently used first): eager
+    banked calls (each reads the chosen experts back to the host once), timed
+    with CUDA events on the stream; hit rate and host-to-device traffic of the
+    paging."""
+    import torch
+    from routed_expert_ffn_fp32_b200 import moe, synth
+    L = ls.host
+    host = moe.Experts(**{f: torch.from_numpy(L["experts"][f]) for f in FIELDS})
+    bank = moe.SlotBank(host, cfg.H, cfg.I, n_slots, device=dev)
+    Wd, bd = router
+    xs = [torch.from_numpy(synth.activations(cfg, 8000 + i, T).view(np.int16)).to(dev)
+          for i in range(16)]
+    shape = moe.shape_of(T, cfg.H, cfg.I, cfg.E, cfg.k)
+    ws = moe.banked_workspace(shape, n_slots, device=dev, stream=stream)
+    y = torch.empty((T, cfg.H), dtype=torch.int16, device=dev)
+    idx = torch.empty((T, cfg.k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, cfg.k), dtype=torch.float32, device=dev)
+    with torch.cuda.stream(stream):
+        for i in range(5):
+            moe.moe_layer_forward_banked(xs[i % 16], Wd, bd, bank, None, shape, y, ws, idx, w,
+                                         stream=stream)
+        stream.synchronize()
+        h0, m0, e0 = bank.stats()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(steps):
+            moe.moe_layer_forward_banked(xs[i % 16], Wd, bd, bank, None, shape, y, ws, idx, w,
+                                         stream=stream)
+        b.record(stream)
+        stream.synchronize()
+    assert moe.moe_get_error(ws, stream) == 0
+    ms = a.elapsed_time(b) / steps
+    h, m, e = (v - v0 for v, v0 in zip(bank.stats(), (h0, m0, e0)))
+    bank.close()
+    h2d = m * expert_bytes(cfg) / steps
+    return {"tokens_per_s": round(T / (ms / 1e3), 1), "ms_per_step": round(ms, 5),
+            "slots": n_slots, "experts": cfg.E, "hit_rate": round(h / max(1, h + m), 4),
+            "h2d_bytes_per_step": int(h2d), "h2d_gbs": round(h2d / (ms / 1e3) / 1e9, 1),
+            "config": workload_config(cfg.with_T(T), T, "exact", "auto", 1),
+            "api": "moe_layer_forward_banked (eager: one host read of the routing per call)"}
 
 
 # ----------------------------------------------------- batch-size sweep ----

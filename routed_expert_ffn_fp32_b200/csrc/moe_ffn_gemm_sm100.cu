@@ -20,15 +20,21 @@
 // re-quantised to MXFP4 along I.  Phase 1: W = down, epilogue writes the
 // float32 expert outputs into `partial` rows (pair index order).
 //
-// CTA roles (192 threads, one persistent CTA per SM):
+// CTA roles (224 threads, one persistent CTA per SM):
 //   warp 0      TMA producer: weight and activation tiles (128-byte swizzle,
-//               no multicast) plus the E8M0 scale bytes, staged by the 32
-//               lanes into the tcgen05 scale-factor atom layout
-//               (byte 16*(r%32) + 4*(r/32%4) + k of a 512-byte atom holds the
-//               scale of row r, K-block k);
+//               no multicast), one arrival with the transaction bytes per
+//               stage;
+//   warp 6      scale producer: the E8M0 scale bytes of each pair of stages
+//               (16 bytes of every row), loaded into registers one pair ahead
+//               and written as whole rows of the tcgen05 scale-factor atom
+//               layout (byte 16*(r%32) + 4*(r/32%4) + k of a 512-byte atom
+//               holds the scale of row r, K-block k); the next work item's
+//               weight-scale block is prefetched into L2;
 //   warp 1      TMEM allocation; lane 0 issues tcgen05.cp (scales -> TMEM)
 //               and tcgen05.mma, and commits stage / accumulator barriers;
 //   warps 2..5  epilogue: tcgen05.ld of their 32-lane TMEM quarter.
+// Each stage's full barrier completes on the tile bytes plus the scale
+// warp's arrival; both producers wait on its empty barrier.
 // Every mbarrier wait is bounded (globaltimer); on expiry the CTA latches
 // MOE_ERR_TIMEOUT in the workspace, drains what it issued and exits.
 #include <cuda.h>
@@ -41,7 +47,7 @@ namespace {
 
 constexpr int kBM = 128;            // weight rows per item (MMA M)
 constexpr int kBKB = 128;           // K bytes per stage (256 FP4 values)
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 224;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
 constexpr int kSmallN = 16;         // token rows of the small activation box
 
@@ -162,6 +168,10 @@ __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap
 }
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// word q (0..3) of a uint4
+__device__ __forceinline__ uint32_t u4_word(const uint4& v, int q) {
+  return q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
 }
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -294,7 +304,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
-      mbar_init(saddr(&full[s]), 2);
+      mbar_init(saddr(&full[s]), 2);  // TMA arrival + scales staged
       mbar_init(saddr(&empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -366,131 +376,167 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int nV = nA + (a.has_shared ? 1 : 0);
   const int n_items = tb.item_off[nV];
 
+  const int my_items = n_items > int(blockIdx.x) ? (n_items - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
+  const int total = my_items * nks;  // stages of this CTA, numbered g = 0..
+
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    // Stages are numbered g = 0.. over this CTA's items (nks stages each).
+    // ------------------------------------------------------- tile producer
     // Items of at most kSmallN tokens load a kSmallN-row activation box
     // instead of BN rows.
-    // The scale words of stage g+1 are loaded into registers while stage g
-    // waits for its slot, so their global latency overlaps the pipeline; the
-    // tile TMAs are issued before the scales are written, and the stage's full
-    // barrier takes two arrivals (TMA transaction + scales staged).
-    constexpr int NB_ROWS = C::NMB * 4;  // 32-row groups of B scale rows
-    int stage = 0;
-    uint32_t phase = 0;
-    uint32_t fills = 0;  // bit s: parity of the last fill of stage s
-    uint32_t used = 0;   // bit s: stage s was filled at least once
-    bool ok = true;
-    const int my_items = n_items > int(blockIdx.x) ? (n_items - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
-    const int total = my_items * nks;
-    Item wn{};
-    int arow_n = 0, brow_n = 0, ks_n = 0;
-    uint32_t sa_n[NPROJ][4][2], sb_n[NB_ROWS][2];
-    auto prepare = [&](int g) {
-      ks_n = g % nks;
-      if (ks_n == 0) {
-        wn = item_of<C::BN>(tb, int(blockIdx.x) + (g / nks) * int(gridDim.x), nV, MT);
-        arow_n = (wn.e >= 0 ? wn.e * ROWS : 0) + wn.mt * kBM;
-        brow_n = wn.row0 + wn.nt * C::BN;
-      }
-      const int sc0 = ks_n * 8;  // first scale byte of the stage
-#pragma unroll
-      for (int p = 0; p < NPROJ; ++p) {
-        const uint8_t* src = (wn.e >= 0 ? a.sa[p] : a.sa_sh[p]);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint8_t* rowp = src + size_t(arow_n + lane + 32 * j) * NSC;
-#pragma unroll
-          for (int at = 0; at < 2; ++at) {
-            const int c = sc0 + 4 * at;
-            sa_n[p][j][at] = c + 4 <= NSC ? __ldg(reinterpret_cast<const uint32_t*>(rowp + c))
-                                          : 0x7f7f7f7fu;
-          }
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t fills = 0;  // bit s: parity of the last fill of stage s
+      uint32_t used = 0;   // bit s: stage s was filled at least once
+      uint64_t pol;
+      asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+      Item w{};
+      int arow = 0, brow = 0;
+      for (int g = 0; g < total; ++g) {
+        const int ks = g % nks;
+        if (ks == 0) {
+          w = item_of<C::BN>(tb, int(blockIdx.x) + (g / nks) * int(gridDim.x), nV, MT);
+          arow = (w.e >= 0 ? w.e * ROWS : 0) + w.mt * kBM;
+          brow = w.row0 + w.nt * C::BN;
         }
-      }
-#pragma unroll
-      for (int j = 0; j < NB_ROWS; ++j) {
-        const int n = lane + 32 * j;
-        const uint8_t* rowp = a.sb + size_t(brow_n + n) * NSC;
-#pragma unroll
-        for (int at = 0; at < 2; ++at) {
-          const int c = sc0 + 4 * at;
-          sb_n[j][at] = (n < wn.nvalid && c + 4 <= NSC)
-                            ? __ldcg(reinterpret_cast<const uint32_t*>(rowp + c))
-                            : 0x7f7f7f7fu;
-        }
-      }
-    };
-    if (total > 0) prepare(0);
-    for (int g = 0; g < total && ok; ++g) {
-      const int ks = ks_n, arow = arow_n, brow = brow_n;
-      const bool routed = wn.e >= 0;
-      const bool small = wn.nvalid <= kSmallN;
-      uint32_t sa[NPROJ][4][2], sb[NB_ROWS][2];
-#pragma unroll
-      for (int p = 0; p < NPROJ; ++p)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          sa[p][j][0] = sa_n[p][j][0];
-          sa[p][j][1] = sa_n[p][j][1];
-        }
-#pragma unroll
-      for (int j = 0; j < NB_ROWS; ++j) {
-        sb[j][0] = sb_n[j][0];
-        sb[j][1] = sb_n[j][1];
-      }
-      if (g + 1 < total) prepare(g + 1);
-      if (!warp_wait(saddr(&empty[stage]), phase ^ 1u, abort_flag, a.err, 100)) {
-        ok = false;
-        break;
-      }
-      unsigned char* st = smem + stage * C::STAGE;
-      unsigned char* sfa = st + NPROJ * C::A_BYTES + C::B_BYTES;
-      unsigned char* sfb = sfa + NPROJ * C::SFA_BYTES;
-      const uint32_t fb = saddr(&full[stage]);
-      if (lane == 0) {
-        uint64_t pol;
-        asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+        const bool routed = w.e >= 0;
+        const bool small = w.nvalid <= kSmallN;
+        if (!mbar_wait(saddr(&empty[stage]), phase ^ 1u, abort_flag, a.err, 100)) break;
+        unsigned char* st = smem + stage * C::STAGE;
+        const uint32_t fb = saddr(&full[stage]);
         mbar_expect_tx(fb, NPROJ * C::A_BYTES + (small ? kSmallN : C::BN) * kBKB);
         tma_load_2d_hint(saddr(st), routed ? &mA0 : &mS0, ks * kBKB, arow, fb, pol);
         if constexpr (NPROJ == 2)
           tma_load_2d_hint(saddr(st + C::A_BYTES), routed ? &mA1 : &mS1, ks * kBKB, arow, fb, pol);
         tma_load_2d(saddr(st + NPROJ * C::A_BYTES), small ? &mBs : &mB, ks * kBKB, brow, fb);
+        fills ^= 1u << stage;  // parity of this fill's phase = bit after toggle ^ 1
+        used |= 1u << stage;
+        if (++stage == C::NS) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
-      // scale words -> atom layout: K atom `at` of row r at at*512 + 16*(r%32) + 4*(r/32%4)
+      // after a give-up, let every tile this thread requested land (bounded)
+      if (*abort_flag) {
+        for (int s = 0; s < C::NS; ++s) {
+          if (!((used >> s) & 1u)) continue;
+          const uint32_t last_parity = ((fills >> s) & 1u) ^ 1u;
+          const unsigned long long t0 = globaltimer();
+          while (!mbar_try(saddr(&full[s]), last_parity) && globaltimer() - t0 < 100000000ull) {
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    // ------------------------------------------------------ scale producer
+    // The stages of an item are taken in pairs (the last one alone when nks
+    // is odd).  Lane l holds rows l, l+32, l+64, l+96 of each operand; word q
+    // of a row's 16 bytes is stage q/2 of the pair, atom q%2.
+    constexpr int NBJ = C::NMB * 4;  // 32-row groups of B scale rows
+    int stage = 0;
+    uint32_t phase = 0;
+    const bool vec16 = (NSC & 15) == 0;  // rows start 16-byte aligned
+    // the weight-scale block of item li of this CTA (128 contiguous rows of
+    // NSC bytes per projection) -> L2, an item ahead of its first use
+    auto prefetch_item = [&](int li) {
+      if (lane != 0 || li >= my_items) return;
+      const Item x = item_of<C::BN>(tb, int(blockIdx.x) + li * int(gridDim.x), nV, MT);
+      const size_t off = (size_t(x.e >= 0 ? x.e * ROWS : 0) + size_t(x.mt) * kBM) * NSC;
+#pragma unroll
+      for (int p = 0; p < NPROJ; ++p)
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"((x.e >= 0 ? a.sa[p] : a.sa_sh[p]) + off),
+                     "r"(uint32_t(kBM * NSC))
+                     : "memory");
+    };
+    Item wn{};
+    int arow_n = 0, brow_n = 0;
+    uint4 sa_n[NPROJ][4], sb_n[NBJ];
+    auto load_pair = [&](int g_n) {
+      const int ks_n = g_n % nks;
+      if (ks_n == 0) {
+        wn = item_of<C::BN>(tb, int(blockIdx.x) + (g_n / nks) * int(gridDim.x), nV, MT);
+        arow_n = (wn.e >= 0 ? wn.e * ROWS : 0) + wn.mt * kBM;
+        brow_n = wn.row0 + wn.nt * C::BN;
+        prefetch_item(g_n / nks + 1);
+      }
+      const int c0 = ks_n * 8;  // first scale byte of the pair
+      // words past the end of a row (the tail of K) read as zero scales:
+      // their K blocks are never multiplied
+      auto row16 = [&](const uint8_t* rowp) {
+        if (vec16 && c0 + 16 <= NSC) return __ldg(reinterpret_cast<const uint4*>(rowp + c0));
+        uint32_t v[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          v[q] = c0 + 4 * q + 4 <= NSC ? __ldg(reinterpret_cast<const uint32_t*>(rowp + c0 + 4 * q)) : 0u;
+        return make_uint4(v[0], v[1], v[2], v[3]);
+      };
+#pragma unroll
+      for (int p = 0; p < NPROJ; ++p) {
+        const uint8_t* src = wn.e >= 0 ? a.sa[p] : a.sa_sh[p];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sa_n[p][j] = row16(src + size_t(arow_n + lane + 32 * j) * NSC);
+      }
+#pragma unroll
+      for (int j = 0; j < NBJ; ++j) {
+        const int n = lane + 32 * j;
+        sb_n[j] = n < wn.nvalid ? row16(a.sb + size_t(brow_n + n) * NSC) : make_uint4(0, 0, 0, 0);
+      }
+    };
+    prefetch_item(0);
+    if (total > 0) load_pair(0);
+    for (int g = 0; g < total;) {
+      const int ks = g % nks;
+      const int npair = ks + 1 < nks ? 2 : 1;
+      uint4 sa[NPROJ][4], sb[NBJ];
 #pragma unroll
       for (int p = 0; p < NPROJ; ++p)
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 4; ++j) sa[p][j] = sa_n[p][j];
 #pragma unroll
-          for (int at = 0; at < 2; ++at)
-            *reinterpret_cast<uint32_t*>(sfa + p * C::SFA_BYTES + at * 512 + 16 * lane + 4 * j) =
-                sa[p][j][at];
-#pragma unroll
-      for (int j = 0; j < NB_ROWS; ++j)
-#pragma unroll
-        for (int at = 0; at < 2; ++at)
-          *reinterpret_cast<uint32_t*>(sfb + at * C::NMB * 512 + (j / 4) * 512 + 16 * lane +
-                                       4 * (j % 4)) = sb[j][at];
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(fb);
-      fills ^= 1u << stage;  // parity of this fill's phase = bit after toggle ^ 1
-      used |= 1u << stage;
+      for (int j = 0; j < NBJ; ++j) sb[j] = sb_n[j];
+      if (g + npair < total) load_pair(g + npair);
+      const int slot0 = stage;
+      const uint32_t phase0 = phase;
       if (++stage == C::NS) {
         stage = 0;
         phase ^= 1u;
       }
-    }
-    // after a give-up, let every tile this warp requested land (bounded)
-    if (*abort_flag && lane == 0) {
-      for (int s = 0; s < C::NS; ++s) {
-        if (!((used >> s) & 1u)) continue;
-        const uint32_t last_parity = ((fills >> s) & 1u) ^ 1u;
-        const unsigned long long t0 = globaltimer();
-        while (!mbar_try(saddr(&full[s]), last_parity) && globaltimer() - t0 < 100000000ull) {
+      const int slot1 = stage;
+      const uint32_t phase1 = phase;
+      if (npair == 2 && ++stage == C::NS) {
+        stage = 0;
+        phase ^= 1u;
+      }
+      if (!warp_wait(saddr(&empty[slot0]), phase0 ^ 1u, abort_flag, a.err, 110)) break;
+      if (npair == 2 && !warp_wait(saddr(&empty[slot1]), phase1 ^ 1u, abort_flag, a.err, 111)) break;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (u == npair) break;
+        unsigned char* sfa = smem + (u ? slot1 : slot0) * C::STAGE + NPROJ * C::A_BYTES + C::B_BYTES;
+        unsigned char* sfb = sfa + NPROJ * C::SFA_BYTES;
+#pragma unroll
+        for (int at = 0; at < 2; ++at) {
+          const int q = 2 * u + at;
+#pragma unroll
+          for (int p = 0; p < NPROJ; ++p)
+            *reinterpret_cast<uint4*>(sfa + p * C::SFA_BYTES + at * 512 + 16 * lane) =
+                make_uint4(u4_word(sa[p][0], q), u4_word(sa[p][1], q), u4_word(sa[p][2], q),
+                           u4_word(sa[p][3], q));
+#pragma unroll
+          for (int mb = 0; mb < C::NMB; ++mb)
+            *reinterpret_cast<uint4*>(sfb + at * C::NMB * 512 + mb * 512 + 16 * lane) =
+                make_uint4(u4_word(sb[4 * mb], q), u4_word(sb[4 * mb + 1], q),
+                           u4_word(sb[4 * mb + 2], q), u4_word(sb[4 * mb + 3], q));
         }
       }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(saddr(&full[slot0]));
+        if (npair == 2) mbar_arrive(saddr(&full[slot1]));
+      }
+      g += npair;
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
@@ -558,7 +604,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     float* tile = epi + q * 32 * 33;  // 32 x 32 transpose tile (phase 0)
@@ -612,16 +658,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           __syncwarp();
         } else {
+          // partial rows of the chunk's 32 tokens: one coalesced load, then
+          // broadcast, so the stores do not wait on index loads one by one
+          const int nl = c0 + lane;
+          int prow_l = 0;
+          if (nl < w.nvalid) {
+            const int r = w.nt * C::BN + nl;
+            prow_l = w.e >= 0 ? __ldg(a.entries + w.row0 + r) : a.T * a.k + r;
+          }
           float o[32];
           tmem_ld32(taddr, o);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const int n = c0 + j;
-            if (n < w.nvalid) {
-              const int r = w.nt * C::BN + n;
-              const int prow = w.e >= 0 ? a.entries[w.row0 + r] : a.T * a.k + r;
-              a.partial[size_t(prow) * a.H + wrow] = o[j];
-            }
+            const int prow = __shfl_sync(kFull, prow_l, j);
+            if (c0 + j < w.nvalid) a.partial[size_t(prow) * a.H + wrow] = o[j];
           }
         }
       }
