@@ -182,6 +182,9 @@ moe_status_t moe_route_topk(const uint16_t* x, const float* w_router, const floa
   a.H = shape.H;
   a.E = shape.E;
   a.k = shape.k;
+  // the workspace past the routing regions holds the router's K-split sums
+  a.lpart = at<float>(ws, L.h);
+  a.lpart_bytes = ws_bytes - L.h;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_route_logits(a, false, s);
   if (e == cudaSuccess) e = launch_topk(a, s);
@@ -338,6 +341,10 @@ moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router, const f
   r.H = shape.H;
   r.E = shape.E;
   r.k = shape.k;
+  // the h / partial regions are free until the expert FFNs: the router's
+  // K-split sums
+  r.lpart = at<float>(ws, L.h);
+  r.lpart_bytes = ws_bytes - L.h;
   if (rp == MOE_PATH_GEMV) {
     r.xh = at<uint16_t>(ws, L.xh);
     r.xexp = at<uint8_t>(ws, L.xexp);

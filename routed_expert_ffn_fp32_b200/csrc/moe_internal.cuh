@@ -335,6 +335,10 @@ struct RouteArgs {
   int* err;
   int has_shared;
   int T, H, E, k;
+  // optional scratch for the prefill router's K-split partial logits
+  // (f32 [splits][T][E]); null: one split, logits written directly
+  float* lpart;
+  size_t lpart_bytes;
 };
 
 struct FfnArgs {

@@ -458,13 +458,16 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_logits(RouteArgs a, int
 }
 
 // Router logits for prefill-sized batches: a 64-token x 64-expert tile per
-// CTA, K in chunks of 32 staged in shared memory (double buffered), each
-// thread a 4 x 4 register tile.  Products of a chunk are summed into a fresh
-// register and chunk sums are added to the running total, so every product
-// meets at most 32 + H/32 + 1 roundings (the bound the parity tests use).
+// CTA over one of S contiguous K ranges (blockIdx.z), K in chunks of 32
+// staged in shared memory (double buffered), each thread a 4 x 4 register
+// tile, two CTAs per SM.  Products of a chunk are summed into a fresh
+// register and chunk sums are added to the running total; with S > 1 the
+// range sums go to lpart[s] and k_topk adds them in order s = 0.., so every
+// product meets at most 32 + H/32 + 1 roundings (the bound the parity tests
+// use).
 constexpr int kTileT = 64, kTileE = 64, kTileK = 32;
 
-__global__ void __launch_bounds__(256) k_route_logits_tiled(RouteArgs a) {
+__global__ void __launch_bounds__(256, 2) k_route_logits_tiled(RouteArgs a, int S) {
   __shared__ __align__(16) float xs[2][kTileK][kTileT + 4];  // [k][token]
   __shared__ __align__(16) float wsm[2][kTileK][kTileE + 4]; // [k][expert]
   pdl_wait();
@@ -473,13 +476,14 @@ __global__ void __launch_bounds__(256) k_route_logits_tiled(RouteArgs a) {
   const int t0 = blockIdx.y * kTileT, e0 = blockIdx.x * kTileE;
   const int ty = tid / 16, tx = tid % 16;  // 4 tokens ty*4.., 4 experts tx*4..
   const int H = a.H;
-  const int nchunks = H / kTileK;
+  const int nchunks = H / kTileK / S;
+  const int kbase = blockIdx.z * nchunks * kTileK;
   // global -> register staging: each thread loads 8 bf16 of x and 8 floats of W
   const int lr = tid / 4, lc = (tid % 4) * 8;  // row (token / expert) and first k
   uint4 xreg;
   float4 wreg0, wreg1;
   auto gload = [&](int ck) {
-    const int k0 = ck * kTileK + lc;
+    const int k0 = kbase + ck * kTileK + lc;
     const int t = t0 + lr, e = e0 + lr;
     xreg = (t < a.T) ? __ldg(reinterpret_cast<const uint4*>(a.x + size_t(t) * H + k0))
                      : make_uint4(0, 0, 0, 0);
@@ -540,6 +544,7 @@ __global__ void __launch_bounds__(256) k_route_logits_tiled(RouteArgs a) {
     if (ck + 1 < nchunks) sstore(buf ^ 1);
     __syncthreads();
   }
+  float* out = S > 1 ? a.lpart + size_t(blockIdx.z) * a.T * a.E : a.logits;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int t = t0 + ty * 4 + i;
@@ -549,19 +554,43 @@ __global__ void __launch_bounds__(256) k_route_logits_tiled(RouteArgs a) {
       const int e = e0 + tx * 4 + j;
       if (e < a.E) {
         float v = acc[i][j];
-        if (a.bias) v += __ldg(a.bias + e);
-        a.logits[size_t(t) * a.E + e] = v;
+        if (S == 1 && a.bias) v += __ldg(a.bias + e);
+        out[size_t(t) * a.E + e] = v;
       }
     }
   }
 }
 
-__global__ void __launch_bounds__(kRouteThreads) k_topk(RouteArgs a) {
+// K splits of the prefill router: the fewest (1, 2, 4, 8) that give every SM
+// about six CTAs, within the scratch and with whole 32-value chunks per split
+int route_splits(const RouteArgs& a) {
+  const long tiles = long((a.E + kTileE - 1) / kTileE) * ((a.T + kTileT - 1) / kTileT);
+  const size_t per = size_t(a.T) * a.E * 4;
+  int S = 1;
+  while (S < 8 && tiles * S < 6L * device_info().sm_count && (a.H / kTileK) % (2 * S) == 0 &&
+         a.lpart != nullptr && size_t(2 * S) * per <= a.lpart_bytes)
+    S *= 2;
+  return S;
+}
+
+__global__ void __launch_bounds__(kRouteThreads) k_topk(RouteArgs a, int S) {
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5;
   const int t = blockIdx.x * (kRouteThreads / 32) + warp;
   if (t >= a.T) return;
+  if (S > 1) {
+    // the logits row: K-range sums added in range order, then the bias
+    float* row = a.logits + size_t(t) * a.E;
+    for (int e = threadIdx.x & 31; e < a.E; e += 32) {
+      const float* p = a.lpart + size_t(t) * a.E + e;
+      float v = p[0];
+      for (int s = 1; s < S; ++s) v += p[size_t(s) * a.T * a.E];
+      if (a.bias) v += __ldg(a.bias + e);
+      row[e] = v;
+    }
+    __syncwarp();
+  }
   dispatch_nv(a.E, [&]<int NV>() {
     topk_warp<NV>(a.logits + size_t(t) * a.E, a.E, a.k, a.idx + size_t(t) * a.k,
                   a.w + size_t(t) * a.k, nullptr);
@@ -599,8 +628,9 @@ static size_t route_smem(int TT, int H) { return size_t(TT) * H * 2 + 8 * TT * 4
 
 cudaError_t launch_route_logits(const RouteArgs& a, bool fuse_tail, cudaStream_t st) {
   if (!fuse_tail && a.T > 32) {
-    dim3 grid((a.E + kTileE - 1) / kTileE, (a.T + kTileT - 1) / kTileT);
-    return launch_pdl(k_route_logits_tiled, grid, dim3(256), 0, st, a);
+    const int S = route_splits(a);
+    dim3 grid((a.E + kTileE - 1) / kTileE, (a.T + kTileT - 1) / kTileT, S);
+    return launch_pdl(k_route_logits_tiled, grid, dim3(256), 0, st, a, S);
   }
   const int TT = a.T <= 1 ? 1 : (a.T <= 2 ? 2 : (a.T <= 4 ? 4 : 8));
   size_t smem = route_smem(TT, a.H);
@@ -633,7 +663,9 @@ size_t route_fused_smem(int T, int H, int E, int k) {
 
 cudaError_t launch_topk(const RouteArgs& a, cudaStream_t st) {
   const int wpb = kRouteThreads / 32;
-  return launch_pdl(k_topk, dim3((a.T + wpb - 1) / wpb), dim3(kRouteThreads), 0, st, a);
+  // the split count the tiled router used (one split below its batch sizes)
+  const int S = a.T > 32 ? route_splits(a) : 1;
+  return launch_pdl(k_topk, dim3((a.T + wpb - 1) / wpb), dim3(kRouteThreads), 0, st, a, S);
 }
 
 cudaError_t launch_bucket(const RouteArgs& a, cudaStream_t st) {
