@@ -90,10 +90,11 @@ typedef int32_t moe_status_t;
 #define MOE_ERR_DEVICE_DATA (-6)
 
 /* Debug switches (moe_workspace_set_limits).  MOE_DEBUG_STARVE_FIRST_WAIT:
- * the first warp of the row-block GEMV's gate/up kernel waits on a stage that
- * no copy fills, so its bounded wait runs out and MOE_ERR_TIMEOUT is latched
- * (the error path of a device-side wait, exercised without any fault); the
- * call's output is then undefined.  For tests only. */
+ * the gate/up kernel leaves its first stage without copies -- on the
+ * row-block GEMV the first warp's, on the tensor-core GEMM the first CTA's --
+ * so the bounded wait on it runs out and MOE_ERR_TIMEOUT is latched (the
+ * error path of a device-side wait, exercised without any fault); the call's
+ * output is then undefined.  For tests only. */
 #define MOE_DEBUG_STARVE_FIRST_WAIT 1u
 
 typedef struct moe_shape {

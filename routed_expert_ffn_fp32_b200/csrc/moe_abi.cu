@@ -182,9 +182,9 @@ moe_status_t moe_route_topk(const uint16_t* x, const float* w_router, const floa
   a.H = shape.H;
   a.E = shape.E;
   a.k = shape.k;
-  // the workspace past the routing regions holds the router's K-split sums
+  // the layout's regions past the routing ones hold the router's K-split sums
   a.lpart = at<float>(ws, L.h);
-  a.lpart_bytes = ws_bytes - L.h;
+  a.lpart_bytes = (ws_bytes < L.total ? ws_bytes : L.total) - L.h;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_route_logits(a, false, s);
   if (e == cudaSuccess) e = launch_topk(a, s);
@@ -211,6 +211,9 @@ moe_status_t moe_bucket(const int32_t* topk_idx, moe_shape_t shape, int32_t* cou
   a.H = shape.H;
   a.E = shape.E;
   a.k = shape.k;
+  // per-chunk counts of the multi-CTA bucket, inside this shape's layout
+  a.lpart = at<float>(ws, L.h);
+  a.lpart_bytes = (ws_bytes < L.total ? ws_bytes : L.total) - L.h;
   return cuda_status(launch_bucket(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -342,9 +345,9 @@ moe_status_t moe_layer_forward(const uint16_t* x, const float* w_router, const f
   r.E = shape.E;
   r.k = shape.k;
   // the h / partial regions are free until the expert FFNs: the router's
-  // K-split sums
+  // K-split sums and the bucket's per-chunk counts
   r.lpart = at<float>(ws, L.h);
-  r.lpart_bytes = ws_bytes - L.h;
+  r.lpart_bytes = L.total - L.h;
   if (rp == MOE_PATH_GEMV) {
     r.xh = at<uint16_t>(ws, L.xh);
     r.xexp = at<uint8_t>(ws, L.xexp);

@@ -48,7 +48,7 @@ namespace {
 constexpr int kBM = 128;            // weight rows per item (MMA M)
 constexpr int kBKB = 128;           // K bytes per stage (256 FP4 values)
 constexpr int kGemmThreads = 224;
-constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
+constexpr unsigned long long kWaitNs = 2000000000ull;  // default bound of a wait: 2 s
 constexpr int kSmallN = 16;         // token rows of the small activation box
 
 template <int PHASE>
@@ -125,15 +125,15 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait; false if it gave up (or another role already did).  Called by
-// one lane; warp_wait() makes the outcome uniform over a warp.
+// Bounded wait (limit_ns); false if it gave up (or another role already
+// did).  Called by one lane; warp_wait() makes the outcome uniform over a warp.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          int* err, int where) {
+                                          int* err, int where, unsigned long long limit_ns) {
   if (mbar_try(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (!mbar_try(bar, parity)) {
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort = 1;
       latch_error(err, MOE_ERR_TIMEOUT, where);
       return false;
@@ -142,9 +142,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return true;
 }
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          int* err, int where) {
+                                          int* err, int where, unsigned long long limit_ns) {
   int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, err, where);
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, err, where, limit_ns);
   return __shfl_sync(kFull, ok, 0) != 0;
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
@@ -335,6 +335,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   pdl_wait();
   pdl_trigger();
+  // the workspace's wait limit (0: the default) and debug switches
+  const unsigned wait_us = __ldg(reinterpret_cast<const unsigned*>(a.err) + 2);
+  const unsigned debug = __ldg(reinterpret_cast<const unsigned*>(a.err) + 3);
+  const unsigned long long wait_ns = wait_us ? wait_us * 1000ull : kWaitNs;
 
   // routing tables -> shared memory (one round of loads)
   Tables tb;
@@ -401,9 +405,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         const bool routed = w.e >= 0;
         const bool small = w.nvalid <= kSmallN;
-        if (!mbar_wait(saddr(&empty[stage]), phase ^ 1u, abort_flag, a.err, 100)) break;
+        if (!mbar_wait(saddr(&empty[stage]), phase ^ 1u, abort_flag, a.err, 100, wait_ns)) break;
         unsigned char* st = smem + stage * C::STAGE;
         const uint32_t fb = saddr(&full[stage]);
+        if (PHASE == 0 && g == 0 && blockIdx.x == 0 && (debug & MOE_DEBUG_STARVE_FIRST_WAIT)) {
+          // debug switch: the first stage gets no tile copies, so the MMA
+          // thread's bounded wait on it runs out
+          if (++stage == C::NS) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          continue;
+        }
         mbar_expect_tx(fb, NPROJ * C::A_BYTES + (small ? kSmallN : C::BN) * kBKB);
         tma_load_2d_hint(saddr(st), routed ? &mA0 : &mS0, ks * kBKB, arow, fb, pol);
         if constexpr (NPROJ == 2)
@@ -508,8 +521,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         stage = 0;
         phase ^= 1u;
       }
-      if (!warp_wait(saddr(&empty[slot0]), phase0 ^ 1u, abort_flag, a.err, 110)) break;
-      if (npair == 2 && !warp_wait(saddr(&empty[slot1]), phase1 ^ 1u, abort_flag, a.err, 111)) break;
+      if (!warp_wait(saddr(&empty[slot0]), phase0 ^ 1u, abort_flag, a.err, 110, wait_ns)) break;
+      if (npair == 2 && !warp_wait(saddr(&empty[slot1]), phase1 ^ 1u, abort_flag, a.err, 111, wait_ns)) break;
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         if (u == npair) break;
@@ -552,11 +565,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int n_mma = ((w.nvalid + 7) / 8) * 8;
         const int buf = local & 1;
         const uint32_t acc_parity = (uint32_t(local >> 1) & 1u) ^ 1u;
-        if (!mbar_wait(saddr(&acc_empty[buf]), acc_parity, abort_flag, a.err, 200)) break;
+        if (!mbar_wait(saddr(&acc_empty[buf]), acc_parity, abort_flag, a.err, 200, wait_ns)) break;
         tc_fence_after();
         const uint32_t tacc = tmem + buf * C::ACC_COLS;
         for (int ks = 0; ks < nks; ++ks) {
-          if (!mbar_wait(saddr(&full[stage]), phase, abort_flag, a.err, 201)) {
+          if (!mbar_wait(saddr(&full[stage]), phase, abort_flag, a.err, 201, wait_ns)) {
             ok = false;
             break;
           }
@@ -612,7 +625,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++local) {
       const Item w = item_of<C::BN>(tb, it, nV, MT);
       const int buf = local & 1;
-      if (!warp_wait(saddr(&acc_full[buf]), uint32_t(local >> 1) & 1u, abort_flag, a.err, 300))
+      if (!warp_wait(saddr(&acc_full[buf]), uint32_t(local >> 1) & 1u, abort_flag, a.err, 300, wait_ns))
         break;
       tc_fence_after();
       const uint32_t tacc = tmem + buf * C::ACC_COLS;

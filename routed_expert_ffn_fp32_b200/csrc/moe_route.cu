@@ -28,6 +28,8 @@
 //   k_bucket: one CTA; counts by shared-memory atomics, exclusive scan, then a
 //     stable placement of each 1024-pair chunk: ranks among equal experts come
 //     from __match_any_sync inside a warp plus per-warp counts of earlier warps.
+//     Batches of more than 2048 pairs take k_bucket_count + k_bucket_place,
+//     one CTA per 2048 pairs, with the same result.
 #include <float.h>
 
 #include "moe_internal.cuh"
@@ -189,6 +191,7 @@ __device__ __forceinline__ void block_scan2(int a, int b, int& ea, int& eb, int&
 }
 
 // counts[] -> offsets[] / plan[] (active experts ascending); also primes cur[].
+// Null outputs are skipped.
 __device__ void offsets_and_plan(const int* cnt, int E, int32_t* counts, int32_t* offsets,
                                  int32_t* plan, int* cur, int* wsum) {
   const int nthreads = blockDim.x, tid = threadIdx.x;
@@ -206,36 +209,27 @@ __device__ void offsets_and_plan(const int* cnt, int E, int32_t* counts, int32_t
     if (counts) counts[e] = c;
     if (offsets) offsets[e] = ex;
     if (cur) cur[e] = ex;
-    if (c > 0) plan[1 + eact++] = e;
+    if (c > 0 && plan) plan[1 + eact++] = e;
     ex += c;
   }
   if (tid == 0) {
     if (offsets) offsets[E] = total;
-    plan[0] = tact;
+    if (plan) plan[0] = tact;
   }
 }
 
-// Stable counting sort of the npairs pairs by expert; block of any size.
-__device__ void bucket_block(const int32_t* idx, int npairs, int E, int32_t* counts,
-                             int32_t* offsets, int32_t* entries, int32_t* plan, int* err,
-                             BucketSmem s) {
+// Stable placement of pairs [p0, p1) in chunks of the block's size: the next
+// free entry of expert e is s.cur[e] (advanced here); ranks among equal
+// experts come from __match_any_sync inside a warp plus per-warp counts of
+// earlier warps (s.hist, zero on entry and on exit).
+__device__ void place_pairs(const int32_t* idx, int p0, int p1, int E, int32_t* entries,
+                            BucketSmem s) {
   const int tid = threadIdx.x, nthreads = blockDim.x;
-  const int lane = tid & 31, warp = tid >> 5, nwarps = nthreads >> 5;
-  for (int e = tid; e < E; e += nthreads) s.cnt[e] = 0;
-  for (int i = tid; i < nwarps * E; i += nthreads) s.hist[i] = 0;
-  __syncthreads();
-  for (int p = tid; p < npairs; p += nthreads) {
-    const int e = idx[p];
-    if (e >= 0 && e < E) atomicAdd(&s.cnt[e], 1);
-    else latch_error(err, MOE_ERR_DEVICE_DATA, p);
-  }
-  __syncthreads();
-  offsets_and_plan(s.cnt, E, counts, offsets, plan, s.cur, s.wsum);
-  __syncthreads();
+  const int lane = tid & 31, warp = tid >> 5;
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int base = 0; base < npairs; base += nthreads) {
+  for (int base = p0; base < p1; base += nthreads) {
     const int p = base + tid;
-    int e = p < npairs ? idx[p] : -1;
+    int e = p < p1 ? idx[p] : -1;
     const bool valid = e >= 0 && e < E;
     const unsigned grp = __match_any_sync(kFull, valid ? e : (E + lane));
     const int rank = __popc(grp & lt_mask);
@@ -254,6 +248,26 @@ __device__ void bucket_block(const int32_t* idx, int npairs, int E, int32_t* cou
     }
     __syncthreads();
   }
+}
+
+// Stable counting sort of the npairs pairs by expert; block of any size.
+__device__ void bucket_block(const int32_t* idx, int npairs, int E, int32_t* counts,
+                             int32_t* offsets, int32_t* entries, int32_t* plan, int* err,
+                             BucketSmem s) {
+  const int tid = threadIdx.x, nthreads = blockDim.x;
+  const int nwarps = nthreads >> 5;
+  for (int e = tid; e < E; e += nthreads) s.cnt[e] = 0;
+  for (int i = tid; i < nwarps * E; i += nthreads) s.hist[i] = 0;
+  __syncthreads();
+  for (int p = tid; p < npairs; p += nthreads) {
+    const int e = idx[p];
+    if (e >= 0 && e < E) atomicAdd(&s.cnt[e], 1);
+    else latch_error(err, MOE_ERR_DEVICE_DATA, p);
+  }
+  __syncthreads();
+  offsets_and_plan(s.cnt, E, counts, offsets, plan, s.cur, s.wsum);
+  __syncthreads();
+  place_pairs(idx, 0, npairs, E, entries, s);
 }
 
 // One-warp stable bucket for small batches (the decode tail): counts by
@@ -605,6 +619,67 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket(RouteArgs a) {
   bucket_block(a.idx, a.T * a.k, a.E, a.counts, a.offsets, a.entries, a.plan, a.err, bs);
 }
 
+// Multi-CTA stable bucket for large batches (two launches).  CTA c owns the
+// pairs [c*kBucketChunk, (c+1)*kBucketChunk).  k_bucket_count: per-CTA counts
+// per expert into gcnt[c][E] (shared-memory atomics).  k_bucket_place: every
+// CTA adds the counts up in CTA order -- totals and the counts of the CTAs
+// before it -- scans the totals into offsets (CTA 0 writes counts, offsets
+// and the plan), and places its pairs stably from offset + earlier CTAs'
+// counts.  The result equals the one-CTA sort's.
+constexpr int kBucketChunk = 2048;
+
+__global__ void __launch_bounds__(kBucketThreads) k_bucket_count(RouteArgs a, int* gcnt) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  pdl_wait();
+  pdl_trigger();
+  int* cnt = reinterpret_cast<int*>(smem);
+  const int npairs = a.T * a.k;
+  const int p0 = blockIdx.x * kBucketChunk, p1 = min(npairs, p0 + kBucketChunk);
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
+    const int e = a.idx[p];
+    if (e >= 0 && e < a.E) atomicAdd(&cnt[e], 1);
+    else latch_error(a.err, MOE_ERR_DEVICE_DATA, p);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) gcnt[size_t(blockIdx.x) * a.E + e] = cnt[e];
+}
+
+__global__ void __launch_bounds__(kBucketThreads) k_bucket_place(RouteArgs a, const int* gcnt) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  pdl_wait();
+  pdl_trigger();
+  BucketSmem bs = bucket_smem(smem, a.E, kBucketThreads / 32);
+  const int npairs = a.T * a.k;
+  const int c = blockIdx.x, nc = gridDim.x;
+  // totals (bs.cnt) and the counts of the CTAs before this one (bs.hist is
+  // still free: it holds the earlier CTAs' sums until the scan)
+  int* before = reinterpret_cast<int*>(bs.hist);
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+    int tot = 0, pre = 0;
+    for (int j = 0; j < nc; ++j) {
+      const int v = gcnt[size_t(j) * a.E + e];
+      if (j < c) pre += v;
+      tot += v;
+    }
+    bs.cnt[e] = tot;
+    before[e] = pre;
+  }
+  __syncthreads();
+  // every CTA scans the totals into its cursors; CTA 0 also writes the
+  // outputs
+  if (c == 0) offsets_and_plan(bs.cnt, a.E, a.counts, a.offsets, a.plan, bs.cur, bs.wsum);
+  else offsets_and_plan(bs.cnt, a.E, nullptr, nullptr, nullptr, bs.cur, bs.wsum);
+  __syncthreads();
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) bs.cur[e] += before[e];
+  __syncthreads();
+  for (int i = threadIdx.x; i < (kBucketThreads / 32) * a.E; i += blockDim.x) bs.hist[i] = 0;
+  __syncthreads();
+  const int p0 = c * kBucketChunk, p1 = min(npairs, p0 + kBucketChunk);
+  place_pairs(a.idx, p0, p1, a.E, a.entries, bs);
+}
+
 // plan[] from caller-provided offsets (component API path).
 __global__ void __launch_bounds__(kBucketThreads) k_plan(RouteArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -670,8 +745,21 @@ cudaError_t launch_topk(const RouteArgs& a, cudaStream_t st) {
 
 cudaError_t launch_bucket(const RouteArgs& a, cudaStream_t st) {
   const size_t smem = bucket_smem_bytes(a.E, kBucketThreads);
-  cudaError_t err =
-      cudaFuncSetAttribute(k_bucket, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  const int npairs = a.T * a.k;
+  const int nc = (npairs + kBucketChunk - 1) / kBucketChunk;
+  const size_t gbytes = size_t(nc) * a.E * 4;
+  cudaError_t err;
+  if (nc > 1 && a.lpart != nullptr && gbytes <= a.lpart_bytes) {
+    // several chunks and scratch for their counts: the two-launch bucket
+    int* gcnt = reinterpret_cast<int*>(a.lpart);
+    err = launch_pdl(k_bucket_count, dim3(nc), dim3(kBucketThreads), size_t(a.E) * 4, st, a, gcnt);
+    if (err != cudaSuccess) return err;
+    err = cudaFuncSetAttribute(k_bucket_place, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (err != cudaSuccess) return err;
+    return launch_pdl(k_bucket_place, dim3(nc), dim3(kBucketThreads), smem, st, a,
+                      static_cast<const int*>(gcnt));
+  }
+  err = cudaFuncSetAttribute(k_bucket, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (err != cudaSuccess) return err;
   return launch_pdl(k_bucket, dim3(1), dim3(kBucketThreads), smem, st, a);
 }

@@ -242,3 +242,32 @@ def test_expired_wait_latches_timeout_and_next_call_recovers():
     assert moe.moe_get_error(ws) == moe.MOE_OK
     ref = O.layer_forward(L["x"], L["W_r"], None, L["experts"], None, cfg.k)
     check_y(bits_np(y), ref)
+
+
+def test_expired_wait_on_tensor_core_path_latches_timeout():
+    """The same on the tcgen05 GEMM: its first CTA's first stage gets no tile
+    copies, the MMA thread's wait on it runs out within the 1 ms limit, the
+    other roles give up too and free TMEM; the next call is correct."""
+    T = 200
+    cfg = _cfg(1024, 512, 16, 4, T, shared=True, bias=True)
+    L = synth.layer(cfg, 6)
+    D = dev_layer(L)
+    shape = moe.shape_of(T, cfg.H, cfg.I, cfg.E, cfg.k)
+    ws = moe.make_workspace(shape, GEMM, MXFP4, True)
+    y = torch.empty((T, cfg.H), dtype=torch.int16, device="cuda")
+    moe.moe_workspace_set_limits(ws, 1000, moe.MOE_DEBUG_STARVE_FIRST_WAIT)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    moe.moe_layer_forward(D["x"], D["W_r"], D["bias"], D["experts"], D["shared"], shape, y, ws,
+                          GEMM, MXFP4)
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 1.0
+    assert moe.moe_get_error(ws) == moe.MOE_ERR_TIMEOUT
+    moe.moe_workspace_set_limits(ws, 0, 0)
+    moe.moe_layer_forward(D["x"], D["W_r"], D["bias"], D["experts"], D["shared"], shape, y, ws,
+                          GEMM, MXFP4)
+    torch.cuda.synchronize()
+    assert moe.moe_get_error(ws) == moe.MOE_OK
+    ref = O.layer_forward(L["x"], L["W_r"], L["bias"], L["experts"], L["shared"], cfg.k,
+                          "mxfp4_act")
+    check_y(bits_np(y), ref)

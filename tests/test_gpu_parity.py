@@ -126,9 +126,16 @@ def test_bucket_bit_exact(T, E, k):
     assert moe.moe_get_error(ws) == 0
 
 
-def test_bucket_bad_index_latches_error():
-    T, E, k = 6, 8, 2
-    idx = np.array([[0, 1], [2, 9], [3, 4], [5, -1], [6, 7], [1, 0]], np.int32)
+@pytest.mark.parametrize("T", [6, 3000])
+def test_bucket_bad_index_latches_error(T):
+    """Out-of-range indices latch MOE_ERR_DEVICE_DATA and are left out; the
+    3000-token batch takes the multi-CTA bucket (6000 pairs, three chunks)."""
+    E, k = 8, 2
+    rng = np.random.default_rng(T)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    idx[1, 1], idx[3, 1] = 9, -1
+    if T > 6:
+        idx[T - 2, 0] = 100
     shape = moe.shape_of(T, 64, 64, E, k)
     ws = moe.make_workspace(shape, moe.MOE_PATH_GEMV)
     counts = torch.empty(E, dtype=torch.int32, device="cuda")
@@ -137,10 +144,17 @@ def test_bucket_bad_index_latches_error():
     moe.moe_bucket(torch.from_numpy(idx).cuda(), shape, counts, offsets, entries, ws)
     assert moe.moe_get_error(ws) == moe.MOE_ERR_DEVICE_DATA
     assert moe.moe_get_error(ws) == 0                       # cleared by the read
-    valid = idx.copy()
-    keep = (valid >= 0) & (valid < E)
+    flat = idx.reshape(-1)
+    keep = (flat >= 0) & (flat < E)
     assert counts.cpu().numpy().sum() == keep.sum()
     assert offsets.cpu().numpy()[-1] == keep.sum()
+    # the valid pairs in stable expert order; the rest of entries untouched
+    pos = np.nonzero(keep)[0]
+    want = pos[np.argsort(flat[pos], kind="stable")]
+    got = entries.cpu().numpy()
+    np.testing.assert_array_equal(got[:keep.sum()], want)
+    assert (got[keep.sum():] == -7).all()
+    np.testing.assert_array_equal(counts.cpu().numpy(), np.bincount(flat[pos], minlength=E))
 
 
 # ------------------------------------------------------------ expert FFN ----
