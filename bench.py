@@ -345,6 +345,9 @@ def roofline_of(cfg, T, r, peaks, uses_tc, record=None) -> dict:
     out = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
            "frac": round(achieved / peaks["hbm_gbs"], 4),
            "traffic": measured_traffic(record, b) if record else None,
+           **({"traffic_source": f"ncu dram__bytes_read.sum + dram__bytes_write.sum of both phases "
+                                 f"(profiles/{record}), scaled by activated bytes"}
+              if record and measured_traffic(record, b) is not None else {}),
            "kernel": "expert FFN call (plan, scaled f16 token rows, gate/up + SwiGLU, down)",
            "peak_source": peaks["source"], "bytes_per_launch": int(b), "launch_ms": round(ms, 5)}
     if uses_tc:
@@ -449,12 +452,11 @@ def run_ours(args, rank, world, local_rank):
     ms = max_over_ranks(r["ms_layer"], dist, dev)
     value = weak_scaling_value(T, world, ms)
     uses_tc = PREC == moe.MOE_ACT_MXFP4 and PATH in (moe.MOE_PATH_GEMM, moe.MOE_PATH_AUTO)
-    record = None if uses_tc else "k_ffn_mma_decode64_t5.json"
+    if not uses_tc:
+        record = "k_ffn_mma_decode64_t5.json"
+    else:
+        record = "k_ffn_gemm_prefill_t2048.json" if cfg.name == synth.PREFILL.name and T == 2048 else None
     roof = roofline_of(cfg, T, r, peaks, uses_tc, record)
-    if roof.get("traffic") is not None:
-        roof["traffic_source"] = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of both "
-                                  "k_ffn_mma phases (profiles/k_ffn_mma_decode64_t5.json), "
-                                  "scaled by activated bytes")
     e2e = e2e_measure(ls, router, cfg, T, PATH, PREC, r, args.steps, args.warmup, stream)
     # route (fused for T <= 32) + gate/up + down + combine; the tensor-core
     # path adds the activation gather and the work-item plan
@@ -510,7 +512,8 @@ def run_extra(ls64, router64, args, stream, dev, peaks):
     pre = synth.PREFILL
     rp = lsf.router(pre)
     for T in (2048, 4096):
-        ex[f"prefill_T{T}"] = entry(lsf, rp, pre, T, A, M, max(10, steps // 4), uses_tc=True)
+        ex[f"prefill_T{T}"] = entry(lsf, rp, pre, T, A, M, max(10, steps // 4), uses_tc=True,
+                                    record="k_ffn_gemm_prefill_t2048.json" if T == 2048 else None)
     ex["sweep"] = sweep_rows(lsf, rp, synth.SWEEP, stream, reps=max(10, steps // 10),
                              variants=("gemv_mxfp4", "gemm_mxfp4"))
     ex["banked_decode64_T5"] = banked_entry(ls64, router64, synth.DECODE64, 5, 32,
@@ -559,7 +562,9 @@ def banked_entry(ls, router, cfg, T, n_slots, steps, stream, dev):
     return {"tokens_per_s": round(T / (ms / 1e3), 1), "ms_per_step": round(ms, 5),
             "slots": n_slots, "experts": cfg.E, "hit_rate": round(h / max(1, h + m), 4),
             "h2d_bytes_per_step": int(h2d), "h2d_gbs": round(h2d / (ms / 1e3) / 1e9, 1),
-            "config": workload_config(cfg.with_T(T), T, "exact", "auto", 1),
+            "config": dict(workload_config(cfg.with_T(T), T, "exact", "auto", 1),
+                           l2=f"{cfg.E} experts in pinned host memory, {n_slots} device slots "
+                              f"({n_slots * expert_bytes(cfg) / 1e9:.2f} GB, larger than L2)"),
             "api": "moe_layer_forward_banked (eager: one host read of the routing per call)"}
 
 
