@@ -471,62 +471,70 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_logits(RouteArgs a, int
   }
 }
 
-// Router logits for prefill-sized batches: a 64-token x 64-expert tile per
+// Router logits for prefill-sized batches: a 128-token x 64-expert tile per
 // CTA over one of S contiguous K ranges (blockIdx.z), K in chunks of 32
-// staged in shared memory (double buffered), each thread a 4 x 4 register
-// tile, two CTAs per SM.  Products of a chunk are summed into a fresh
-// register and chunk sums are added to the running total; with S > 1 the
-// range sums go to lpart[s] and k_topk adds them in order s = 0.., so every
-// product meets at most 32 + H/32 + 1 roundings (the bound the parity tests
-// use).
-constexpr int kTileT = 64, kTileE = 64, kTileK = 32;
+// staged in shared memory (double buffered, dynamic), each thread an
+// 8-token x 4-expert register tile, two CTAs per SM.  Products of a chunk are
+// summed into a fresh register and chunk sums are added to the running total;
+// with S > 1 the range sums go to lpart[s] and k_topk adds them in order
+// s = 0.., so every product meets at most 32 + H/32 + 1 roundings (the bound
+// the parity tests use).
+constexpr int kTileT = 128, kTileE = 64, kTileK = 32;
+constexpr int kXPitch = kTileT + 4, kWPitch = kTileE + 4;  // floats per k row
+constexpr size_t kTiledSmem = size_t(2) * kTileK * (kXPitch + kWPitch) * 4;
 
 __global__ void __launch_bounds__(256, 2) k_route_logits_tiled(RouteArgs a, int S) {
-  __shared__ __align__(16) float xs[2][kTileK][kTileT + 4];  // [k][token]
-  __shared__ __align__(16) float wsm[2][kTileK][kTileE + 4]; // [k][expert]
+  extern __shared__ __align__(16) float tsm[];
+  float* xs = tsm;                              // [2][kTileK][kXPitch]  [k][token]
+  float* wsm = tsm + 2 * kTileK * kXPitch;      // [2][kTileK][kWPitch]  [k][expert]
   pdl_wait();
   pdl_trigger();
   const int tid = threadIdx.x;
   const int t0 = blockIdx.y * kTileT, e0 = blockIdx.x * kTileE;
-  const int ty = tid / 16, tx = tid % 16;  // 4 tokens ty*4.., 4 experts tx*4..
+  const int ty = tid / 16, tx = tid % 16;  // tokens ty*8.., experts tx*4..
   const int H = a.H;
   const int nchunks = H / kTileK / S;
   const int kbase = blockIdx.z * nchunks * kTileK;
-  // global -> register staging: each thread loads 8 bf16 of x and 8 floats of W
-  const int lr = tid / 4, lc = (tid % 4) * 8;  // row (token / expert) and first k
-  uint4 xreg;
+  // global -> register staging of a chunk: 16 bf16 of one token row and 8
+  // floats of one expert row per thread
+  const int xr = tid / 2, xc = (tid % 2) * 16;  // token, first k
+  const int wr = tid / 4, wc = (tid % 4) * 8;   // expert, first k
+  uint4 xreg0, xreg1;
   float4 wreg0, wreg1;
   auto gload = [&](int ck) {
-    const int k0 = kbase + ck * kTileK + lc;
-    const int t = t0 + lr, e = e0 + lr;
-    xreg = (t < a.T) ? __ldg(reinterpret_cast<const uint4*>(a.x + size_t(t) * H + k0))
-                     : make_uint4(0, 0, 0, 0);
+    const int k0 = kbase + ck * kTileK;
+    const int t = t0 + xr, e = e0 + wr;
+    if (t < a.T) {
+      const uint4* px = reinterpret_cast<const uint4*>(a.x + size_t(t) * H + k0 + xc);
+      xreg0 = __ldg(px);
+      xreg1 = __ldg(px + 1);
+    } else {
+      xreg0 = xreg1 = make_uint4(0, 0, 0, 0);
+    }
     if (e < a.E) {
-      wreg0 = __ldg(reinterpret_cast<const float4*>(a.w_router + size_t(e) * H + k0));
-      wreg1 = __ldg(reinterpret_cast<const float4*>(a.w_router + size_t(e) * H + k0 + 4));
+      const float4* pw = reinterpret_cast<const float4*>(a.w_router + size_t(e) * H + k0 + wc);
+      wreg0 = __ldg(pw);
+      wreg1 = __ldg(pw + 1);
     } else {
       wreg0 = wreg1 = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   };
   auto sstore = [&](int buf) {
-    const uint32_t xw[4] = {xreg.x, xreg.y, xreg.z, xreg.w};
+    float* xb = xs + buf * kTileK * kXPitch;
+    float* wb = wsm + buf * kTileK * kWPitch;
+    const uint32_t xw[8] = {xreg0.x, xreg0.y, xreg0.z, xreg0.w, xreg1.x, xreg1.y, xreg1.z, xreg1.w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      xs[buf][lc + 2 * j][lr] = bf16_bits_to_f32(xw[j] & 0xffffu);
-      xs[buf][lc + 2 * j + 1][lr] = bf16_bits_to_f32(xw[j] >> 16);
+    for (int j = 0; j < 8; ++j) {
+      xb[(xc + 2 * j) * kXPitch + xr] = bf16_bits_to_f32(xw[j] & 0xffffu);
+      xb[(xc + 2 * j + 1) * kXPitch + xr] = bf16_bits_to_f32(xw[j] >> 16);
     }
-    wsm[buf][lc + 0][lr] = wreg0.x;
-    wsm[buf][lc + 1][lr] = wreg0.y;
-    wsm[buf][lc + 2][lr] = wreg0.z;
-    wsm[buf][lc + 3][lr] = wreg0.w;
-    wsm[buf][lc + 4][lr] = wreg1.x;
-    wsm[buf][lc + 5][lr] = wreg1.y;
-    wsm[buf][lc + 6][lr] = wreg1.z;
-    wsm[buf][lc + 7][lr] = wreg1.w;
-  };
-  float acc[4][4];
+    const float wv[8] = {wreg0.x, wreg0.y, wreg0.z, wreg0.w, wreg1.x, wreg1.y, wreg1.z, wreg1.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+    for (int j = 0; j < 8; ++j) wb[(wc + j) * kWPitch + wr] = wv[j];
+  };
+  float acc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
   gload(0);
@@ -535,24 +543,27 @@ __global__ void __launch_bounds__(256, 2) k_route_logits_tiled(RouteArgs a, int 
   for (int ck = 0; ck < nchunks; ++ck) {
     const int buf = ck & 1;
     if (ck + 1 < nchunks) gload(ck + 1);
-    float part[4][4];
+    const float* xb = xs + buf * kTileK * kXPitch + ty * 8;
+    const float* wb = wsm + buf * kTileK * kWPitch + tx * 4;
+    float part[8][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) part[i][j] = 0.f;
-#pragma unroll 8
+#pragma unroll 4
     for (int k = 0; k < kTileK; ++k) {
-      const float4 xv = *reinterpret_cast<const float4*>(&xs[buf][k][ty * 4]);
-      const float4 wv = *reinterpret_cast<const float4*>(&wsm[buf][k][tx * 4]);
-      const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
-      const float wa[4] = {wv.x, wv.y, wv.z, wv.w};
+      const float4 xa = *reinterpret_cast<const float4*>(xb + k * kXPitch);
+      const float4 xb4 = *reinterpret_cast<const float4*>(xb + k * kXPitch + 4);
+      const float4 wv = *reinterpret_cast<const float4*>(wb + k * kWPitch);
+      const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb4.x, xb4.y, xb4.z, xb4.w};
+      const float ww[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(xa[i], wa[j], part[i][j]);
+        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(xv[i], ww[j], part[i][j]);
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
     if (ck + 1 < nchunks) sstore(buf ^ 1);
@@ -560,8 +571,8 @@ __global__ void __launch_bounds__(256, 2) k_route_logits_tiled(RouteArgs a, int 
   }
   float* out = S > 1 ? a.lpart + size_t(blockIdx.z) * a.T * a.E : a.logits;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = t0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const int t = t0 + ty * 8 + i;
     if (t >= a.T) continue;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -575,16 +586,36 @@ __global__ void __launch_bounds__(256, 2) k_route_logits_tiled(RouteArgs a, int 
   }
 }
 
-// K splits of the prefill router: the fewest (1, 2, 4, 8) that give every SM
+// K splits of the prefill router: the fewest (1, 2, 4, 8, 16) that give every SM
 // about six CTAs, within the scratch and with whole 32-value chunks per split
 int route_splits(const RouteArgs& a) {
   const long tiles = long((a.E + kTileE - 1) / kTileE) * ((a.T + kTileT - 1) / kTileT);
   const size_t per = size_t(a.T) * a.E * 4;
   int S = 1;
-  while (S < 8 && tiles * S < 6L * device_info().sm_count && (a.H / kTileK) % (2 * S) == 0 &&
+  while (S < 16 && tiles * S < 6L * device_info().sm_count && (a.H / kTileK) % (2 * S) == 0 &&
          a.lpart != nullptr && size_t(2 * S) * per <= a.lpart_bytes)
     S *= 2;
   return S;
+}
+
+// The logits row of token t from the router's S K-range sums: all S loads of
+// a logit first, then the sums added in range order, then the bias (one warp).
+template <int S>
+__device__ __forceinline__ void sum_splits(const RouteArgs& a, int t) {
+  float* row = a.logits + size_t(t) * a.E;
+  const size_t stride = size_t(a.T) * a.E;
+#pragma unroll 2
+  for (int e = threadIdx.x & 31; e < a.E; e += 32) {
+    const float* p = a.lpart + size_t(t) * a.E + e;
+    float v[S];
+#pragma unroll
+    for (int s = 0; s < S; ++s) v[s] = p[s * stride];
+    float acc = v[0];
+#pragma unroll
+    for (int s = 1; s < S; ++s) acc += v[s];
+    if (a.bias) acc += __ldg(a.bias + e);
+    row[e] = acc;
+  }
 }
 
 __global__ void __launch_bounds__(kRouteThreads) k_topk(RouteArgs a, int S) {
@@ -594,14 +625,11 @@ __global__ void __launch_bounds__(kRouteThreads) k_topk(RouteArgs a, int S) {
   const int t = blockIdx.x * (kRouteThreads / 32) + warp;
   if (t >= a.T) return;
   if (S > 1) {
-    // the logits row: K-range sums added in range order, then the bias
-    float* row = a.logits + size_t(t) * a.E;
-    for (int e = threadIdx.x & 31; e < a.E; e += 32) {
-      const float* p = a.lpart + size_t(t) * a.E + e;
-      float v = p[0];
-      for (int s = 1; s < S; ++s) v += p[size_t(s) * a.T * a.E];
-      if (a.bias) v += __ldg(a.bias + e);
-      row[e] = v;
+    switch (S) {
+      case 2: sum_splits<2>(a, t); break;
+      case 4: sum_splits<4>(a, t); break;
+      case 8: sum_splits<8>(a, t); break;
+      default: sum_splits<16>(a, t); break;
     }
     __syncwarp();
   }
@@ -705,7 +733,11 @@ cudaError_t launch_route_logits(const RouteArgs& a, bool fuse_tail, cudaStream_t
   if (!fuse_tail && a.T > 32) {
     const int S = route_splits(a);
     dim3 grid((a.E + kTileE - 1) / kTileE, (a.T + kTileT - 1) / kTileT, S);
-    return launch_pdl(k_route_logits_tiled, grid, dim3(256), 0, st, a, S);
+    cudaError_t err = cudaFuncSetAttribute(k_route_logits_tiled,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           int(kTiledSmem));
+    if (err != cudaSuccess) return err;
+    return launch_pdl(k_route_logits_tiled, grid, dim3(256), kTiledSmem, st, a, S);
   }
   const int TT = a.T <= 1 ? 1 : (a.T <= 2 ? 2 : (a.T <= 4 ? 4 : 8));
   size_t smem = route_smem(TT, a.H);
