@@ -163,7 +163,11 @@ MOE_API moe_status_t moe_workspace_set_limits(void* ws, uint32_t wait_us, uint32
 /* Router, softmax, top-k and renormalisation.
  * logits[t,e] = sum_h x[t,h] W_r[e,h] + bias[e] in float32 (bias may be NULL);
  * topk_idx/topk_w as described above.  logits_out [T, E] float32 may be NULL.
- * Ties of equal float32 logits go to the lower expert index. */
+ * Ties of equal float32 logits go to the lower expert index.  ws must hold the
+ * routing part of moe_workspace_bytes(shape, ...); batches above 32 tokens
+ * split the router's dot products over up to 16 K ranges when ws also covers
+ * the shape's later regions (their sums are added in range order, so every
+ * product meets at most 32 + H/32 + 1 float32 roundings). */
 MOE_API moe_status_t moe_route_topk(const uint16_t* x, const float* w_router,
                             const float* bias, moe_shape_t shape,
                             float* logits_out, int32_t* topk_idx,
@@ -172,7 +176,9 @@ MOE_API moe_status_t moe_route_topk(const uint16_t* x, const float* w_router,
 
 /* Stable counting sort of the T*k (token, slot) pairs by expert: writes
  * counts [E], offsets [E+1] and entries [T*k] (layouts above).  An index
- * outside [0, E) latches MOE_ERR_DEVICE_DATA and the pair is dropped. */
+ * outside [0, E) latches MOE_ERR_DEVICE_DATA and the pair is dropped.  Above
+ * 2048 pairs, when ws covers the shape's later regions, one CTA per 2048
+ * pairs sorts its chunk (same result). */
 MOE_API moe_status_t moe_bucket(const int32_t* topk_idx, moe_shape_t shape,
                         int32_t* counts, int32_t* offsets, int32_t* entries,
                         void* ws, size_t ws_bytes, void* stream);
