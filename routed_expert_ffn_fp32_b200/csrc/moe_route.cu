@@ -11,14 +11,16 @@
 // which equals softmax over all E followed by renormalisation over the k.
 //
 // Kernels
-//   k_route_logits<TT>: one CTA per (2 experts, TT tokens).  Eight warps:
-//     warp w takes expert (w / 4) of the pair and the w % 4 quarter of H; each
+//   k_route_logits<TT>: one CTA per (2 experts, 1 token) or per (1 expert,
+//     TT > 1 tokens).  Eight warps: with two experts warp w takes expert w / 4
+//     and the w % 4 quarter of H, with one expert the w-th eighth of H; each
 //     lane streams float4 router rows and keeps TT float32 partial sums.  The
 //     bf16 token rows sit in shared memory; the f16 copy of the token rows
 //     for the row-block GEMV is written from there by all CTAs of a token tile,
-//     32 values per thread.  Every product meets at most
-//     H/128 + 9 roundings (lane chain, 5 shuffle levels, 3 quarter sums, the
-//     bias), the bound the parity tests use for near-ties.
+//     32 values per thread.  Every product meets at most H/128 + 9 roundings
+//     (lane chain, 5 shuffle levels, 3 sums of the warps' parts -- a chain of
+//     quarters or a tree of eighths -- and the bias), the bound the parity
+//     tests use for near-ties.
 //     With fuse_tail the CTA that finishes last (arrival counter in the
 //     workspace, reset to zero by that CTA) runs top-k (a warp per token) and
 //     a one-warp bucket for the whole batch, so a decode step routes in one
@@ -342,9 +344,13 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_logits(RouteArgs a, int
   const int nt = min(TT, a.T - t0);
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);                  // [TT][H] bf16
   float* red = reinterpret_cast<float*>(smem + size_t(TT) * H * 2);  // [8][TT]
-  const int e = blockIdx.x * 2 + (warp >> 2);
-  const int quarter = warp & 3;
-  const int qlen = H / 4;  // multiple of 8
+  // experts per CTA: two for single-token tiles (eight warps split each row
+  // in quarters), else one (eighths)
+  constexpr int EPC = TT == 1 ? 2 : 1;
+  constexpr int PARTS = 8 / EPC;
+  const int e = blockIdx.x * EPC + warp / PARTS;
+  const int quarter = warp % PARTS;  // this warp's part of the row
+  const int qlen = H / PARTS;        // multiple of 4
   const float* wrow = a.w_router + size_t(e < a.E ? e : 0) * H + quarter * qlen;
   // the first eight float4 of this lane's router row go out before the token
   // rows are staged, so the two loads overlap
@@ -438,12 +444,18 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_logits(RouteArgs a, int
     for (int t = 0; t < TT; ++t) red[warp * TT + t] = acc[t];
   }
   __syncthreads();
-  if (tid < 2 * TT) {
+  if (tid < EPC * TT) {
     const int pe = tid / TT, t = tid % TT;
-    const int ee = blockIdx.x * 2 + pe;
+    const int ee = blockIdx.x * EPC + pe;
     if (ee < a.E && t < nt) {
-      const float* r = red + (pe * 4) * TT + t;
-      float s = ((r[0] + r[TT]) + r[2 * TT]) + r[3 * TT];
+      const float* r = red + (pe * PARTS) * TT + t;
+      float s;
+      if constexpr (PARTS == 4) {
+        s = ((r[0] + r[TT]) + r[2 * TT]) + r[3 * TT];
+      } else {
+        s = ((r[0] + r[TT]) + (r[2 * TT] + r[3 * TT])) +
+            ((r[4 * TT] + r[5 * TT]) + (r[6 * TT] + r[7 * TT]));
+      }
       if (a.bias) s += __ldg(a.bias + ee);
       a.logits[size_t(t0 + t) * a.E + ee] = s;
     }
@@ -745,7 +757,7 @@ cudaError_t launch_route_logits(const RouteArgs& a, bool fuse_tail, cudaStream_t
     const size_t tail = align_up16(size_t(a.T) * a.k * 4) + size_t(a.E) * 8;
     smem = smem > tail ? smem : tail;
   }
-  dim3 grid((a.E + 1) / 2, (a.T + TT - 1) / TT);
+  dim3 grid(TT == 1 ? (a.E + 1) / 2 : a.E, (a.T + TT - 1) / TT);
   cudaError_t err = cudaSuccess;
   auto go = [&](auto kern) {
     err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
