@@ -127,8 +127,9 @@ typedef struct moe_mxfp4_experts {
 /* Activation precision of the expert projections.  EXACT: the bf16 token
  * rows and the fp32 SwiGLU output enter the projections without quantisation
  * (the pages' quality mode, "ds4-ssd" README, "Experimental Pro Support":
- * --quality / --no-int8), with float32 accumulation.  On the CUDA-core path
- * for T <= 512 (the row-block GEMV, whose products run on f16 tensor-core
+ * --quality / --no-int8), with float32 accumulation.  A single token takes
+ * the K-split GEMV (float32 products throughout).  On the CUDA-core path for
+ * 2 <= T <= 512 (the row-block GEMV, whose products run on f16 tensor-core
  * operands) token row t enters as f16 values of x * 2^-s_t, its largest
  * magnitude scaled into [1, 2) and 2^s_t applied to the sums: every bf16
  * value within 2^-17 of its row's largest magnitude is exact, smaller ones
