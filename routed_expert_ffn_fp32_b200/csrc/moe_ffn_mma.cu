@@ -1205,10 +1205,7 @@ bool lane_supported(const moe_shape_t& s) {
   const int smem = LaneCfg<2>::SMEM > LaneCfg<1>::SMEM ? LaneCfg<2>::SMEM : LaneCfg<1>::SMEM;
   // the per-expert tables hold 256 routed experts and the shared one
   const bool prefix_fits = s.E + 2 <= kPfxMax;
-  // a single token takes the K-split GEMV: with one token per expert every
-  // row block is split over many warps here, and the whole layer measured
-  // faster there (decode64 36.7 -> 33.1 us)
-  return s.T >= 2 && s.T <= kLaneMaxT && s.H % kAtomVals == 0 && s.I % kAtomVals == 0 && prefix_fits &&
+  return s.T <= kLaneMaxT && s.H % kAtomVals == 0 && s.I % kAtomVals == 0 && prefix_fits &&
          device_info().max_smem_optin >= smem;
 }
 
