@@ -295,6 +295,9 @@ class SlotBank:
 
 def moe_layer_forward_banked(x, w_router, bias, bank: SlotBank, shared, shape, y, ws, topk_idx,
                              topk_w, path=MOE_PATH_AUTO, precision=MOE_ACT_EXACT, stream=None):
+    """The layer over a slot bank: routes, reads the chosen experts back once
+    (one synchronisation of the stream), makes them resident and runs the
+    FFNs over the bank's slots.  topk_idx / topk_w receive the routing."""
     _check(load_library().moe_layer_forward_banked(_p(x), _p(w_router), _p(bias), bank.handle,
                                                    _ex(shared), shape, path, precision, _p(y),
                                                    _p(topk_idx), _p(topk_w), _p(ws), ws.numel(),
@@ -303,6 +306,7 @@ def moe_layer_forward_banked(x, w_router, bias, bank: SlotBank, shared, shape, y
 
 def banked_workspace(shape, n_slots, path=MOE_PATH_AUTO, precision=MOE_ACT_EXACT,
                      has_shared=False, device="cuda", stream=None) -> torch.Tensor:
+    """A zeroed workspace for moe_layer_forward_banked with n_slots slots."""
     n = int(load_library().moe_layer_forward_banked_workspace_bytes(shape, n_slots, path, precision,
                                                                     int(has_shared)))
     if n == 0:
