@@ -114,7 +114,13 @@ def ep_layer_forward(x, w_router, bias, shard: ExpertShard, shape, y, ws, group=
         import torch.distributed as dist
     y32, idx, w = ep_partial(x, w_router, bias, shard, shape, ws, path, precision, stream, lib)
     if dist.is_initialized() and dist.get_world_size(group) > 1:
-        dist.all_reduce(y32, op=dist.ReduceOp.SUM, group=group)
+        # the collective orders itself after the work of torch's current
+        # stream: make it the stream the library calls ran on
+        if stream is not None and y32.is_cuda:
+            with torch.cuda.stream(stream):
+                dist.all_reduce(y32, op=dist.ReduceOp.SUM, group=group)
+        else:
+            dist.all_reduce(y32, op=dist.ReduceOp.SUM, group=group)
     ep_finish(y32, y, stream, lib)
     return idx, w
 
