@@ -22,6 +22,7 @@ the single-device layer up to float32 rounding of that sum.
 """
 from __future__ import annotations
 
+import contextlib
 import dataclasses
 
 import torch
@@ -69,12 +70,24 @@ class ExpertShard:
         return cls(e0, e1, local, shared if rank == shared_rank else None)
 
 
+def _on(stream):
+    """torch's current stream set to ``stream`` (when given), so the scratch
+    tensors below are allocated, and freed, in the order of the library calls
+    that use them."""
+    return torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+
+
 def ep_partial(x, w_router, bias, shard: ExpertShard, shape, ws, path=moe.MOE_PATH_AUTO,
                precision=moe.MOE_ACT_EXACT, stream=None, lib=moe):
     """Steps 1-4 on this rank: the float32 [T, H] partial output of the pairs
     whose expert this rank holds (plus the shared expert on its rank), and the
     routing (topk_idx, topk_w).  ``ws`` must cover moe_workspace_bytes of the
     full shape and of the local one (see ep_workspace_bytes)."""
+    with _on(stream):
+        return _ep_partial(x, w_router, bias, shard, shape, ws, path, precision, stream, lib)
+
+
+def _ep_partial(x, w_router, bias, shard, shape, ws, path, precision, stream, lib):
     T, H, I, E, k = shape.T, shape.H, shape.I, shape.E, shape.k
     dev = x.device
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
@@ -116,10 +129,7 @@ def ep_layer_forward(x, w_router, bias, shard: ExpertShard, shape, y, ws, group=
     if dist.is_initialized() and dist.get_world_size(group) > 1:
         # the collective orders itself after the work of torch's current
         # stream: make it the stream the library calls ran on
-        if stream is not None and y32.is_cuda:
-            with torch.cuda.stream(stream):
-                dist.all_reduce(y32, op=dist.ReduceOp.SUM, group=group)
-        else:
+        with _on(stream if y32.is_cuda else None):
             dist.all_reduce(y32, op=dist.ReduceOp.SUM, group=group)
     ep_finish(y32, y, stream, lib)
     return idx, w
