@@ -1,5 +1,6 @@
 """Expert parallelism on the CPU: the shard ranges, and the orchestration of
-ep_layer_forward over two gloo ranks on 127.0.0.1.
+ep_layer_forward over two and four gloo ranks on 127.0.0.1 (with four, one
+rank holds no expert).
 
 The per-rank compute steps are a CPU stand-in built from the fp64 oracle
 (test code only, passed as ``lib``): this checks the host logic of the
@@ -136,12 +137,16 @@ def _rank(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_match_single_device_oracle():
+@pytest.mark.parametrize("world,ranges", [
+    (2, [(0, 8), (8, 12)]),
+    # the last rank holds no expert: its partial is zero, the sum unchanged
+    (4, [(0, 4), (4, 8), (8, 12), (12, 12)]),
+])
+def test_gloo_ranks_match_single_device_oracle(world, ranges):
     sys.path.insert(0, ROOT)
     import oracle as O
     from helpers import check_y
     from routed_expert_ffn_fp32_b200 import synth
-    world = 2
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -152,7 +157,7 @@ def test_two_gloo_ranks_match_single_device_oracle():
     for p in procs:
         p.join(timeout=120)
         assert p.exitcode == 0
-    assert [(r[1], r[2]) for r in res] == [(0, 8), (8, 12)]
+    assert [(r[1], r[2]) for r in res] == ranges
     cfg = synth.LayerConfig("ep", 128, 64, 12, 3, 6, 0.05, 1.0, True)
     L = synth.layer(cfg, 41)
     ref = O.layer_forward(L["x"], L["W_r"], L["bias"], L["experts"], L["shared"], cfg.k)
